@@ -1,0 +1,570 @@
+// C ABI of libbytecross: model handle, workspace layout, the decode-step
+// launch sequence, single-kernel entry points and the byte account.
+#include "../../include/bytecross.h"
+#include "common.cuh"
+#include "kernels.h"
+
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+#include <algorithm>
+#include <string>
+
+using namespace bc;
+
+// ------------------------------------------------------------------ errors
+static thread_local std::string g_err;
+
+static bc_status fail(bc_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+static bc_status fail(bc_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+static bc_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(BC_ECUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define BC_CUDA(call, where)                              \
+  do {                                                    \
+    cudaError_t e_ = (call);                              \
+    if (e_ != cudaSuccess) return cuda_fail(e_, where);   \
+  } while (0)
+
+extern "C" const char* bc_last_error(void) { return g_err.c_str(); }
+
+extern "C" const char* bc_status_string(bc_status s) {
+  switch (s) {
+    case BC_OK: return "ok";
+    case BC_EINVAL: return "invalid argument";
+    case BC_ENOMEM: return "buffer too small";
+    case BC_ECAPACITY: return "KV capacity exceeded";
+    case BC_ECUDA: return "CUDA error";
+    case BC_ETIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+// ------------------------------------------------------------------ config and layout
+static bool check_config(const bc_config* c, std::string* why) {
+  if (!c) { *why = "null config"; return false; }
+  if (c->n_layers < 1 || c->hidden < 1 || c->intermediate < 1 || c->vocab < 1 || c->max_ctx < 1) {
+    *why = "dimensions must be positive"; return false;
+  }
+  if (c->head_dim != 64 && c->head_dim != 128) { *why = "head_dim must be 64 or 128"; return false; }
+  if (c->n_kv_heads < 1 || c->n_heads % c->n_kv_heads != 0 || c->n_heads / c->n_kv_heads > 8) {
+    *why = "n_heads must be 1..8 times n_kv_heads"; return false;
+  }
+  if (c->n_heads * c->head_dim != c->hidden) { *why = "n_heads * head_dim must equal hidden"; return false; }
+  if (c->page != kPage) { *why = "page must be 16"; return false; }
+  if (c->hidden % kColTile || c->intermediate % kColTile) {
+    *why = "hidden and intermediate must be multiples of 256"; return false;
+  }
+  if (c->intermediate > kMaxSelect || c->hidden > kMaxSelect) { *why = "hidden/intermediate above 16384"; return false; }
+  if ((c->max_ctx + kPage - 1) / kPage > kMaxSelect) { *why = "max_ctx above 262144"; return false; }
+  if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) { *why = "rms_eps > 0 and rope_theta > 1 required"; return false; }
+  return true;
+}
+
+struct Layout {
+  size_t x, xf, logits, xn, qkv, q, attn, xn2, gu, h, xo;    // f32 (per-layer ones are [L][..])
+  size_t sel_qkv, sel_o, sel_gu, sel_d;                         // int32 [L][..]
+  size_t pscore, pages;                                         // [L][Hkv][Pmax]
+  size_t part_o, part_ml, gemv_part, counters;
+  size_t total;
+  int nqkv, hq, Pmax, max_dout;
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static Layout make_layout(const bc_config* c) {
+  Layout y;
+  const size_t L = c->n_layers, d = c->hidden, f = c->intermediate;
+  y.hq = c->n_heads * c->head_dim;
+  y.nqkv = (c->n_heads + 2 * c->n_kv_heads) * c->head_dim;
+  y.Pmax = (c->max_ctx + kPage - 1) / kPage;
+  y.max_dout = (int)std::max<size_t>(std::max<size_t>(y.nqkv, d), 2 * f);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align256(o + bytes); return at; };
+  y.x = take(4 * d);
+  y.xf = take(4 * d);
+  y.logits = take(4 * (size_t)c->vocab);
+  y.xn = take(4 * L * d);
+  y.qkv = take(4 * L * y.nqkv);
+  y.q = take(4 * L * y.hq);
+  y.attn = take(4 * L * y.hq);
+  y.xn2 = take(4 * L * d);
+  y.gu = take(4 * L * 2 * f);
+  y.h = take(4 * L * f);
+  y.xo = take(4 * L * d);
+  y.sel_qkv = take(4 * L * d);
+  y.sel_o = take(4 * L * y.hq);
+  y.sel_gu = take(4 * L * d);
+  y.sel_d = take(4 * L * f);
+  y.pscore = take(4 * L * c->n_kv_heads * (size_t)y.Pmax);
+  y.pages = take(4 * L * c->n_kv_heads * (size_t)y.Pmax);
+  y.part_o = take(4 * (size_t)c->n_heads * kMaxSplits * c->head_dim);
+  y.part_ml = take(4 * (size_t)c->n_heads * kMaxSplits * 2);
+  y.gemv_part = take(4 * (size_t)kGemvMaxChunks * y.max_dout);
+  y.counters = take(4 * 4 * (size_t)(y.max_dout / kColTile));
+  y.total = o;
+  return y;
+}
+
+extern "C" size_t bc_kv_pool_bytes(const bc_config* c) {
+  std::string why;
+  if (!check_config(c, &why)) return 0;
+  const size_t Pmax = (c->max_ctx + kPage - 1) / kPage;
+  return (size_t)c->n_layers * c->n_kv_heads * Pmax * 2 * kPage * c->head_dim * 2;
+}
+
+extern "C" size_t bc_meta_pool_bytes(const bc_config* c) {
+  std::string why;
+  if (!check_config(c, &why)) return 0;
+  const size_t Pmax = (c->max_ctx + kPage - 1) / kPage;
+  return (size_t)c->n_layers * c->n_kv_heads * Pmax * 2 * c->head_dim * 2;
+}
+
+extern "C" size_t bc_workspace_bytes(const bc_config* c) {
+  std::string why;
+  if (!check_config(c, &why)) return 0;
+  return make_layout(c).total;
+}
+
+// ------------------------------------------------------------------ model
+struct bc_model {
+  bc_config cfg;
+  bc_weights w;
+  __nv_bfloat16* kv;
+  __nv_bfloat16* meta;
+  char* ws;
+  size_t ws_bytes;
+  cudaStream_t stream;
+  Layout lay;
+  int n;               // cached tokens
+  int sms;
+  long long launches;  // kernels launched so far
+  // what the last step left in the traces
+  int last_k[4];       // kept channels per site (0 = no selection)
+  int last_P, last_K;  // pages after the append, kept pages (0 = no selection)
+};
+
+template <typename T>
+static T* at(const bc_model* m, size_t off) { return reinterpret_cast<T*>(m->ws + off); }
+
+static int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+extern "C" bc_status bc_model_create(const bc_config* cfg, const bc_weights* w, void* kv_pool,
+                                     void* meta_pool, void* workspace, size_t ws_bytes,
+                                     void* stream, bc_model** out) {
+  std::string why;
+  if (!out) return fail(BC_EINVAL, "out is null");
+  *out = nullptr;
+  if (!check_config(cfg, &why)) return fail(BC_EINVAL, "bad config: %s", why.c_str());
+  if (!w || !w->embed || !w->lm_head || !w->final_norm || !w->attn_norm || !w->mlp_norm ||
+      !w->wqkv_t || !w->wo_t || !w->wgu_t || !w->wd_t)
+    return fail(BC_EINVAL, "null weight pointer");
+  if (!kv_pool || !meta_pool || !workspace) return fail(BC_EINVAL, "null pool or workspace");
+  if (((uintptr_t)kv_pool | (uintptr_t)meta_pool | (uintptr_t)workspace) & 255)
+    return fail(BC_EINVAL, "pools and workspace must be 256-byte aligned");
+  Layout lay = make_layout(cfg);
+  if (ws_bytes < lay.total)
+    return fail(BC_ENOMEM, "workspace has %zu bytes, needs %zu", ws_bytes, lay.total);
+  bc_model* m = new bc_model();
+  m->cfg = *cfg;
+  m->w = *w;
+  m->kv = static_cast<__nv_bfloat16*>(kv_pool);
+  m->meta = static_cast<__nv_bfloat16*>(meta_pool);
+  m->ws = static_cast<char*>(workspace);
+  m->ws_bytes = ws_bytes;
+  m->stream = static_cast<cudaStream_t>(stream);
+  m->lay = lay;
+  m->n = 0;
+  m->sms = device_sms();
+  m->launches = 0;
+  memset(m->last_k, 0, sizeof m->last_k);
+  m->last_P = m->last_K = 0;
+  cudaError_t e = cudaMemsetAsync(m->ws + lay.counters, 0, 4 * 4 * (size_t)(lay.max_dout / kColTile), m->stream);
+  if (e != cudaSuccess) {
+    delete m;
+    return cuda_fail(e, "bc_model_create: clearing counters");
+  }
+  *out = m;
+  return BC_OK;
+}
+
+extern "C" bc_status bc_model_destroy(bc_model* m) {
+  delete m;
+  return BC_OK;
+}
+
+extern "C" bc_status bc_set_stream(bc_model* m, void* stream) {
+  if (!m) return fail(BC_EINVAL, "null model");
+  m->stream = static_cast<cudaStream_t>(stream);
+  return BC_OK;
+}
+
+extern "C" int bc_kv_length(const bc_model* m) { return m ? m->n : -1; }
+
+extern "C" long long bc_launch_count(const bc_model* m) { return m ? m->launches : -1; }
+
+extern "C" bc_status bc_kv_reset(bc_model* m, int n_ctx) {
+  if (!m) return fail(BC_EINVAL, "null model");
+  if (n_ctx < 0 || n_ctx > m->n) return fail(BC_EINVAL, "reset to %d outside [0, %d]", n_ctx, m->n);
+  m->n = n_ctx;
+  return BC_OK;
+}
+
+extern "C" bc_status bc_kv_append(bc_model* m, const void* k, const void* v, int n_tokens) {
+  if (!m) return fail(BC_EINVAL, "null model");
+  if (n_tokens < 0) return fail(BC_EINVAL, "n_tokens < 0");
+  if (n_tokens == 0) return BC_OK;
+  if (!k || !v) return fail(BC_EINVAL, "null k or v");
+  if ((long long)m->n + n_tokens > m->cfg.max_ctx)
+    return fail(BC_ECAPACITY, "append of %d tokens to %d exceeds max_ctx %d", n_tokens, m->n, m->cfg.max_ctx);
+  KvAppendArgs a;
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.n_new = n_tokens;
+  a.n0 = m->n;
+  a.L = m->cfg.n_layers;
+  a.Hkv = m->cfg.n_kv_heads;
+  a.hd = m->cfg.head_dim;
+  a.Pmax = m->lay.Pmax;
+  a.pool = m->kv;
+  a.meta = m->meta;
+  BC_CUDA(launch_kv_append(a, m->stream, true), "bc_kv_append");
+  m->launches += 2;
+  m->n += n_tokens;
+  return BC_OK;
+}
+
+static int keep_count(float ratio, int n) {
+  const double v = ceil((double)ratio * n - 1e-9);
+  return (int)std::max(1.0, std::min((double)n, v));
+}
+
+static bc_status check_step(const bc_model* m, bc_mode mode, float rp, float rkv, int sinks,
+                            int recent, int page) {
+  if (!m) return fail(BC_EINVAL, "null model");
+  if (mode < BC_DENSE || mode > BC_BOTH) return fail(BC_EINVAL, "bad mode %d", (int)mode);
+  if (page != m->cfg.page) return fail(BC_EINVAL, "page %d differs from the model's %d", page, m->cfg.page);
+  if (!(rp > 0.f && rp <= 1.f)) return fail(BC_EINVAL, "rp %g outside (0, 1]", rp);
+  if (!(rkv > 0.f && rkv <= 1.f)) return fail(BC_EINVAL, "rkv %g outside (0, 1]", rkv);
+  if (sinks < 0 || recent < 1) return fail(BC_EINVAL, "sinks must be >= 0 and recent >= 1");
+  if (m->n + 1 > m->cfg.max_ctx) return fail(BC_ECAPACITY, "KV cache full (%d tokens)", m->n);
+  return BC_OK;
+}
+
+static cudaError_t step_select(bc_model* m, int prep, int n, bool sel, int k, const float* v,
+                               const __nv_bfloat16* gain, const __nv_bfloat16* emb, float* x_out,
+                               float* out, int* idx) {
+  SelectArgs s;
+  s.prep = prep;
+  s.n = n;
+  s.k = k;
+  s.do_select = sel ? 1 : 0;
+  s.v = v;
+  s.gain = gain;
+  s.eps = m->cfg.rms_eps;
+  s.embed_row = emb;
+  s.x_out = x_out;
+  s.out = out;
+  s.idx = idx;
+  return launch_select(s, m->stream, true);
+}
+
+static cudaError_t step_gemv(bc_model* m, int site, const __nv_bfloat16* W, int d_in, int d_out,
+                             const float* x, const int* idx, int k, int epi, float* y,
+                             float* y_copy, const QkvEpilogue* qe) {
+  GemvArgs g;
+  g.W = W;
+  g.d_in = d_in;
+  g.d_out = d_out;
+  g.x = x;
+  g.idx = idx;
+  g.k = k;
+  gemv_plan(k, d_out, m->sms, kGemvMaxChunks, &g.chunk, &g.n_chunks);
+  g.partial = at<float>(m, m->lay.gemv_part);
+  g.counters = at<unsigned>(m, m->lay.counters) + site * (m->lay.max_dout / kColTile);
+  g.epi = epi;
+  g.y = y;
+  g.y_copy = y_copy;
+  if (qe) g.qkv = *qe;
+  else memset(&g.qkv, 0, sizeof g.qkv);
+  return launch_gemv(g, m->stream, true);
+}
+
+static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, float rkv, int sinks,
+                              int recent, float* logits) {
+  const bc_config& c = m->cfg;
+  const Layout& y = m->lay;
+  const bool act = mode == BC_ACT || mode == BC_BOTH;
+  const bool kvs = mode == BC_KV || mode == BC_BOTH;
+  const int L = c.n_layers, d = c.hidden, f = c.intermediate, hd = c.head_dim;
+  const int Hq = c.n_heads, Hkv = c.n_kv_heads, G = Hq / Hkv;
+  const int hq = y.hq, nqkv = y.nqkv, Pmax = y.Pmax;
+  const int pos = m->n, n_tok = pos + 1;
+  const int P = (n_tok + kPage - 1) / kPage;
+  int K = P;
+  if (kvs) {
+    const int sink_end = std::min(sinks, P), rec_begin = std::max(P - recent, 0);
+    const int n_forced = sink_end + (P - std::max(rec_begin, sink_end));
+    const int want = (int)std::min<double>(P, ceil((double)rkv * P - 1e-9));
+    K = std::max(n_forced, want);
+  }
+  const int k_qkv = act ? keep_count(rp, d) : d;
+  const int k_o = act ? keep_count(rp, hq) : hq;
+  const int k_gu = act ? keep_count(rp, d) : d;
+  const int k_d = act ? keep_count(rp, f) : f;
+
+  const __nv_bfloat16* emb = static_cast<const __nv_bfloat16*>(m->w.embed) + (size_t)token * d;
+  const __nv_bfloat16* attn_norm = static_cast<const __nv_bfloat16*>(m->w.attn_norm);
+  const __nv_bfloat16* mlp_norm = static_cast<const __nv_bfloat16*>(m->w.mlp_norm);
+  const __nv_bfloat16* wqkv = static_cast<const __nv_bfloat16*>(m->w.wqkv_t);
+  const __nv_bfloat16* wo = static_cast<const __nv_bfloat16*>(m->w.wo_t);
+  const __nv_bfloat16* wgu = static_cast<const __nv_bfloat16*>(m->w.wgu_t);
+  const __nv_bfloat16* wd = static_cast<const __nv_bfloat16*>(m->w.wd_t);
+  float* x = at<float>(m, y.x);
+  const size_t kv_layer = (size_t)Hkv * Pmax * 2 * kPage * hd;
+  const size_t meta_layer = (size_t)Hkv * Pmax * 2 * hd;
+
+  int splits, pps;
+  attn_plan(K, Hkv, m->sms, &splits, &pps);
+
+  for (int l = 0; l < L; ++l) {
+    float* xn = at<float>(m, y.xn) + (size_t)l * d;
+    float* qkv = at<float>(m, y.qkv) + (size_t)l * nqkv;
+    float* q = at<float>(m, y.q) + (size_t)l * hq;
+    float* attn = at<float>(m, y.attn) + (size_t)l * hq;
+    float* xn2 = at<float>(m, y.xn2) + (size_t)l * d;
+    float* gu = at<float>(m, y.gu) + (size_t)l * 2 * f;
+    float* hmid = at<float>(m, y.h) + (size_t)l * f;
+    float* xo = at<float>(m, y.xo) + (size_t)l * d;
+    int* s_qkv = at<int>(m, y.sel_qkv) + (size_t)l * d;
+    int* s_o = at<int>(m, y.sel_o) + (size_t)l * hq;
+    int* s_gu = at<int>(m, y.sel_gu) + (size_t)l * d;
+    int* s_d = at<int>(m, y.sel_d) + (size_t)l * f;
+    float* pscore = at<float>(m, y.pscore) + (size_t)l * Hkv * Pmax;
+    int* pages = at<int>(m, y.pages) + (size_t)l * Hkv * Pmax;
+    __nv_bfloat16* kvl = m->kv + l * kv_layer;
+    __nv_bfloat16* metal = m->meta + l * meta_layer;
+
+    // attention block
+    BC_CUDA(step_select(m, l == 0 ? PREP_EMBED_NORM : PREP_NORM, d, act, k_qkv, x,
+                        attn_norm + (size_t)l * d, emb, x, xn, s_qkv), "select qkv");
+    QkvEpilogue qe;
+    qe.Hq = Hq;
+    qe.Hkv = Hkv;
+    qe.hd = hd;
+    qe.pos = pos;
+    qe.Pmax = Pmax;
+    qe.rope_theta = c.rope_theta;
+    qe.q_out = q;
+    qe.kv_layer = kvl;
+    qe.meta_layer = metal;
+    BC_CUDA(step_gemv(m, 0, wqkv + (size_t)l * d * nqkv, d, nqkv, xn, act ? s_qkv : nullptr, k_qkv,
+                      EPI_QKV, qkv, nullptr, &qe), "gemv qkv");
+    if (kvs) {
+      PageScoreArgs ps{q, metal, Hkv, G, hd, Pmax, P, pscore};
+      BC_CUDA(launch_page_scores(ps, m->stream, true), "page scores");
+      PageSelectArgs pl{pscore, Hkv, Pmax, P, K, sinks, recent, pages};
+      BC_CUDA(launch_page_select(pl, m->stream, true), "page select");
+    }
+    AttnArgs aa;
+    aa.q = q;
+    aa.kv = kvl;
+    aa.pages = kvs ? pages : nullptr;
+    aa.Hkv = Hkv;
+    aa.G = G;
+    aa.hd = hd;
+    aa.Pmax = Pmax;
+    aa.n_pages = K;
+    aa.n_tok = n_tok;
+    aa.splits = splits;
+    aa.pages_per_split = pps;
+    aa.part_o = at<float>(m, y.part_o);
+    aa.part_ml = at<float>(m, y.part_ml);
+    aa.out = attn;
+    BC_CUDA(launch_attention(aa, m->stream, true), "attention");
+    if (act)
+      BC_CUDA(step_select(m, PREP_NONE, hq, true, k_o, attn, nullptr, nullptr, nullptr, nullptr, s_o),
+              "select o");
+    BC_CUDA(step_gemv(m, 1, wo + (size_t)l * hq * d, hq, d, attn, act ? s_o : nullptr, k_o, EPI_RESID,
+                      x, nullptr, nullptr), "gemv o");
+    // feed-forward block
+    BC_CUDA(step_select(m, PREP_NORM, d, act, k_gu, x, mlp_norm + (size_t)l * d, nullptr, nullptr,
+                        xn2, s_gu), "select gate/up");
+    BC_CUDA(step_gemv(m, 2, wgu + (size_t)l * d * 2 * f, d, 2 * f, xn2, act ? s_gu : nullptr, k_gu,
+                      EPI_STORE, gu, nullptr, nullptr), "gemv gate/up");
+    BC_CUDA(step_select(m, PREP_SWIGLU, f, act, k_d, gu, nullptr, nullptr, nullptr, hmid, s_d),
+            "select down");
+    BC_CUDA(step_gemv(m, 3, wd + (size_t)l * f * d, f, d, hmid, act ? s_d : nullptr, k_d, EPI_RESID,
+                      x, xo, nullptr), "gemv down");
+  }
+  float* xf = at<float>(m, y.xf);
+  BC_CUDA(step_select(m, PREP_NORM, d, false, d, x, static_cast<const __nv_bfloat16*>(m->w.final_norm),
+                      nullptr, nullptr, xf, nullptr), "final norm");
+  LmHeadArgs lm{static_cast<const __nv_bfloat16*>(m->w.lm_head), c.vocab, d, xf, logits};
+  BC_CUDA(launch_lmhead(lm, m->sms, m->stream, true), "lm head");
+
+  // launches: per layer norm/select, q/k/v, attention + combine, o, norm/select,
+  // gate/up, swiglu/select, down; the kv branch adds scores and page select,
+  // the projection branch the select of the attention output; then the
+  // final norm and the LM head
+  m->launches += (long long)L * (9 + (kvs ? 2 : 0) + (act ? 1 : 0)) + 2;
+  m->n = n_tok;
+  m->last_k[0] = act ? k_qkv : 0;
+  m->last_k[1] = act ? k_o : 0;
+  m->last_k[2] = act ? k_gu : 0;
+  m->last_k[3] = act ? k_d : 0;
+  m->last_P = P;
+  m->last_K = kvs ? K : 0;
+  return BC_OK;
+}
+
+extern "C" bc_status bc_decode_step(bc_model* m, int token, bc_mode mode, float rp, float rkv,
+                                    int sinks, int recent, int page, float* logits) {
+  bc_status s = check_step(m, mode, rp, rkv, sinks, recent, page);
+  if (s != BC_OK) return s;
+  if (!logits) return fail(BC_EINVAL, "null logits");
+  if (token < 0 || token >= m->cfg.vocab) return fail(BC_EINVAL, "token %d outside the vocabulary", token);
+  return enqueue_step(m, token, mode, rp, rkv, sinks, recent, logits);
+}
+
+extern "C" bc_status bc_decode_step_host(bc_model* m, int token, bc_mode mode, float rp, float rkv,
+                                         int sinks, int recent, int page, float* logits_host) {
+  bc_status s = check_step(m, mode, rp, rkv, sinks, recent, page);
+  if (s != BC_OK) return s;
+  if (!logits_host) return fail(BC_EINVAL, "null logits");
+  if (token < 0 || token >= m->cfg.vocab) return fail(BC_EINVAL, "token %d outside the vocabulary", token);
+  float* dev = at<float>(m, m->lay.logits);
+  s = enqueue_step(m, token, mode, rp, rkv, sinks, recent, dev);
+  if (s != BC_OK) return s;
+  BC_CUDA(cudaMemcpyAsync(logits_host, dev, sizeof(float) * m->cfg.vocab, cudaMemcpyDeviceToHost, m->stream),
+          "bc_decode_step_host: copy logits");
+  BC_CUDA(cudaStreamSynchronize(m->stream), "bc_decode_step_host: sync");
+  return BC_OK;
+}
+
+extern "C" bc_status bc_trace(const bc_model* m, int layer, bc_trace_kind kind, const void** ptr,
+                              int* count, int* stride) {
+  if (!m || !ptr || !count) return fail(BC_EINVAL, "null argument");
+  const bc_config& c = m->cfg;
+  const Layout& y = m->lay;
+  if (layer < 0 || layer >= c.n_layers) return fail(BC_EINVAL, "layer %d out of range", layer);
+  const int d = c.hidden, f = c.intermediate, hq = y.hq;
+  size_t off = 0;
+  int n = 0, st = 0;
+  switch (kind) {
+    case BC_TRACE_XN: off = y.xn + 4ull * layer * d; n = d; break;
+    case BC_TRACE_SEL_QKV: off = y.sel_qkv + 4ull * layer * d; n = m->last_k[0]; break;
+    case BC_TRACE_Q: off = y.q + 4ull * layer * hq; n = hq; break;
+    case BC_TRACE_ATTN: off = y.attn + 4ull * layer * hq; n = hq; break;
+    case BC_TRACE_SEL_O: off = y.sel_o + 4ull * layer * hq; n = m->last_k[1]; break;
+    case BC_TRACE_XN2: off = y.xn2 + 4ull * layer * d; n = d; break;
+    case BC_TRACE_SEL_GU: off = y.sel_gu + 4ull * layer * d; n = m->last_k[2]; break;
+    case BC_TRACE_H: off = y.h + 4ull * layer * f; n = f; break;
+    case BC_TRACE_SEL_D: off = y.sel_d + 4ull * layer * f; n = m->last_k[3]; break;
+    case BC_TRACE_X: off = y.xo + 4ull * layer * d; n = d; break;
+    case BC_TRACE_PAGE_SCORES:
+      off = y.pscore + 4ull * layer * c.n_kv_heads * y.Pmax; n = m->last_K ? m->last_P : 0; st = y.Pmax; break;
+    case BC_TRACE_PAGES:
+      off = y.pages + 4ull * layer * c.n_kv_heads * y.Pmax; n = m->last_K; st = y.Pmax; break;
+    case BC_TRACE_QKV: off = y.qkv + 4ull * layer * y.nqkv; n = y.nqkv; break;
+    default: return fail(BC_EINVAL, "bad trace kind %d", (int)kind);
+  }
+  *ptr = m->ws + off;
+  *count = n;
+  if (stride) *stride = st;
+  return BC_OK;
+}
+
+// ------------------------------------------------------------------ single kernels
+extern "C" size_t bc_gemv_scratch_bytes(int d_out) {
+  if (d_out <= 0 || d_out % kColTile) return 0;
+  return align256(4ull * kGemvMaxChunks * d_out) + align256(4ull * (d_out / kColTile));
+}
+
+extern "C" bc_status bc_gemv(const void* W, int d_in, int d_out, const float* x, const int* idx, int k,
+                             float* y, void* scratch, size_t scratch_bytes, void* stream) {
+  if (!W || !x || !y || !scratch) return fail(BC_EINVAL, "null pointer");
+  if (d_in <= 0 || d_out <= 0 || d_out % kColTile) return fail(BC_EINVAL, "d_out must be a positive multiple of 256");
+  if (k < 1 || k > d_in || (!idx && k != d_in)) return fail(BC_EINVAL, "k must be in [1, d_in] (= d_in without idx)");
+  if (scratch_bytes < bc_gemv_scratch_bytes(d_out)) return fail(BC_ENOMEM, "scratch too small");
+  GemvArgs g;
+  g.W = static_cast<const __nv_bfloat16*>(W);
+  g.d_in = d_in;
+  g.d_out = d_out;
+  g.x = x;
+  g.idx = idx;
+  g.k = k;
+  gemv_plan(k, d_out, device_sms(), kGemvMaxChunks, &g.chunk, &g.n_chunks);
+  g.partial = static_cast<float*>(scratch);
+  g.counters = reinterpret_cast<unsigned*>(static_cast<char*>(scratch) + align256(4ull * kGemvMaxChunks * d_out));
+  g.epi = EPI_STORE;
+  g.y = y;
+  g.y_copy = nullptr;
+  memset(&g.qkv, 0, sizeof g.qkv);
+  BC_CUDA(launch_gemv(g, static_cast<cudaStream_t>(stream), true), "bc_gemv");
+  return BC_OK;
+}
+
+extern "C" bc_status bc_select_topk(const float* v, int n, int k, int* idx, void* stream) {
+  if (!v || !idx) return fail(BC_EINVAL, "null pointer");
+  if (n < 1 || n > kMaxSelect || k < 1 || k > n) return fail(BC_EINVAL, "need 1 <= k <= n <= 16384");
+  SelectArgs s;
+  memset(&s, 0, sizeof s);
+  s.prep = PREP_NONE;
+  s.n = n;
+  s.k = k;
+  s.do_select = 1;
+  s.v = v;
+  s.idx = idx;
+  BC_CUDA(launch_select(s, static_cast<cudaStream_t>(stream), true), "bc_select_topk");
+  return BC_OK;
+}
+
+extern "C" size_t bc_attention_scratch_bytes(int n_q_heads, int head_dim) {
+  if (n_q_heads <= 0 || head_dim <= 0) return 0;
+  return align256(4ull * n_q_heads * kMaxSplits * head_dim) + align256(4ull * n_q_heads * kMaxSplits * 2);
+}
+
+extern "C" bc_status bc_attention(const float* q, const void* kv, int n_kv_heads, int group, int head_dim,
+                                  int Pmax, const int* pages, int n_pages, int n_tok, float* out,
+                                  void* scratch, size_t scratch_bytes, void* stream) {
+  if (!q || !kv || !out || !scratch) return fail(BC_EINVAL, "null pointer");
+  if (head_dim != 64 && head_dim != 128) return fail(BC_EINVAL, "head_dim must be 64 or 128");
+  if (n_kv_heads < 1 || group < 1 || group > 8) return fail(BC_EINVAL, "bad head counts");
+  if (n_tok < 1 || n_pages < 1 || Pmax < n_pages || (n_tok + kPage - 1) / kPage > Pmax)
+    return fail(BC_EINVAL, "bad page counts");
+  if (!pages && n_pages != (n_tok + kPage - 1) / kPage) return fail(BC_EINVAL, "without a page list n_pages must cover n_tok");
+  if (scratch_bytes < bc_attention_scratch_bytes(n_kv_heads * group, head_dim)) return fail(BC_ENOMEM, "scratch too small");
+  AttnArgs a;
+  a.q = q;
+  a.kv = static_cast<const __nv_bfloat16*>(kv);
+  a.pages = pages;
+  a.Hkv = n_kv_heads;
+  a.G = group;
+  a.hd = head_dim;
+  a.Pmax = Pmax;
+  a.n_pages = n_pages;
+  a.n_tok = n_tok;
+  attn_plan(n_pages, n_kv_heads, device_sms(), &a.splits, &a.pages_per_split);
+  a.part_o = static_cast<float*>(scratch);
+  a.part_ml = reinterpret_cast<float*>(static_cast<char*>(scratch) + align256(4ull * n_kv_heads * group * kMaxSplits * head_dim));
+  a.out = out;
+  BC_CUDA(launch_attention(a, static_cast<cudaStream_t>(stream), true), "bc_attention");
+  return BC_OK;
+}

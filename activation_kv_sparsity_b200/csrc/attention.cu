@@ -1,0 +1,266 @@
+// Split-K flash-decode attention over a page list: the one attention kernel
+// of every mode.  The ByteCross README ("Overview": "One attention kernel for
+// every mode"; FAQ: a masked dense baseline inflates KV speedups about
+// fivefold) insists that dense and sparse modes read the cache through the
+// same split-K kernel; here dense mode is simply the full page list.
+//
+// Layout: the pages of one (layer, kv head) are 2*16*hd bf16 each, the 16
+// keys then the 16 values (8 KiB at hd = 128).  CTA (split, kv head) walks a
+// contiguous slice of the page list; its 4 warps take every 4th page.
+//
+// Per page a warp runs the two products on the tensor cores with
+// mma.m16n8k16 (bf16 in, fp32 accumulate).  The A operand rows 0..7 carry the
+// G <= 8 query heads of the group rounded to bf16 ("hi"), rows 8..15 the
+// rounding residues ("lo"), so S = S_hi + S_lo keeps about 16 significant
+// bits of the fp32 query; the softmax weights P are split the same way for
+// P*V.  Keys are loaded straight into B fragments: lane (g, t) reads 32
+// consecutive dims of key rows g and g+8, and the contraction dims are
+// permuted consistently in A and B, which leaves the dot products unchanged.
+// Value fragments are transposed in registers with movmatrix.  Each lane
+// ends with its head row's output over hd/4 consecutive dims.
+//
+// Partials (m, l, o) per (query head, split) use base-2 logits; the combine
+// kernel merges them: o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+#include "common.cuh"
+#include "kernels.h"
+
+#include <algorithm>
+
+namespace bc {
+
+constexpr int kAttnWarps = 4;
+
+__device__ __forceinline__ void mma16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t transpose8x8(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// hi/lo bf16 split of two floats: hi = (bf16(x0), bf16(x1)), lo = residues.
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+  hi = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+  lo = pack_bf16x2(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
+}
+
+template <int HD>
+__global__ void __launch_bounds__(kAttnWarps * 32) k_attn(AttnArgs a) {
+  constexpr int KSTEPS = HD / 16;   // k16 steps of q.k
+  constexpr int NBLK = HD / 8;      // n8 blocks of p.v
+  constexpr int DPL = HD / 4;       // dims per lane
+  constexpr int U4 = DPL / 8;       // 16-byte vectors per lane and row
+  constexpr int PAGE_ELEMS = 2 * kPage * HD;
+
+  __shared__ float s_o[kAttnWarps][8][HD];
+  __shared__ float s_m[kAttnWarps][8], s_l[kAttnWarps][8];
+
+  const int split = blockIdx.x, h = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int G = a.G;
+
+  pdl_wait();
+  pdl_trigger();
+
+  // A fragments of the queries, pre-scaled to base-2 logits
+  const float qscale = 1.4426950408889634f * rsqrtf((float)HD);
+  uint32_t qa[KSTEPS][4];
+  {
+    const float* qrow = a.q + (size_t)(h * G + g) * HD + t * DPL;
+    #pragma unroll
+    for (int s = 0; s < KSTEPS; ++s) {
+      float q0 = 0.f, q1 = 0.f, q2 = 0.f, q3 = 0.f;
+      if (g < G) {
+        q0 = qrow[4 * s] * qscale;
+        q1 = qrow[4 * s + 1] * qscale;
+        q2 = qrow[4 * s + 2] * qscale;
+        q3 = qrow[4 * s + 3] * qscale;
+      }
+      split2(q0, q1, qa[s][0], qa[s][1]);
+      split2(q2, q3, qa[s][2], qa[s][3]);
+    }
+  }
+
+  float o[NBLK][4];
+  #pragma unroll
+  for (int b = 0; b < NBLK; ++b) o[b][0] = o[b][1] = o[b][2] = o[b][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+
+  const int i_begin = split * a.pages_per_split;
+  const int i_end = min(a.n_pages, i_begin + a.pages_per_split);
+  const __nv_bfloat16* head_base = a.kv + (size_t)h * a.Pmax * PAGE_ELEMS;
+  const int* plist = a.pages ? a.pages + (size_t)h * a.Pmax : nullptr;
+
+  for (int i = i_begin + warp; i < i_end; i += kAttnWarps) {
+    const int page = plist ? plist[i] : i;
+    const int nxt = i + kAttnWarps;
+    if (lane == 0 && nxt < i_end) {
+      const int pn = plist ? plist[nxt] : nxt;
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                   :: "l"(head_base + (size_t)pn * PAGE_ELEMS), "r"(PAGE_ELEMS * 2) : "memory");
+    }
+    const __nv_bfloat16* pk = head_base + (size_t)page * PAGE_ELEMS + t * DPL;
+    const __nv_bfloat16* pv = pk + kPage * HD;
+    uint4 k0[U4], k1[U4], v0[U4], v1[U4];
+    #pragma unroll
+    for (int u = 0; u < U4; ++u) {
+      k0[u] = ld_stream(pk + g * HD + 8 * u);
+      k1[u] = ld_stream(pk + (g + 8) * HD + 8 * u);
+      v0[u] = ld_stream(pv + g * HD + 8 * u);
+      v1[u] = ld_stream(pv + (g + 8) * HD + 8 * u);
+    }
+    const int valid = min(kPage, a.n_tok - page * kPage);
+    if (g >= valid) {
+      #pragma unroll
+      for (int u = 0; u < U4; ++u) v0[u] = make_uint4(0, 0, 0, 0);
+    }
+    if (g + 8 >= valid) {
+      #pragma unroll
+      for (int u = 0; u < U4; ++u) v1[u] = make_uint4(0, 0, 0, 0);
+    }
+    const uint32_t* kr0 = reinterpret_cast<const uint32_t*>(k0);
+    const uint32_t* kr1 = reinterpret_cast<const uint32_t*>(k1);
+    const uint32_t* vr0 = reinterpret_cast<const uint32_t*>(v0);
+    const uint32_t* vr1 = reinterpret_cast<const uint32_t*>(v1);
+
+    // logits of tokens 0-7 (c0) and 8-15 (c1): rows g = hi, g+8 = lo
+    float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+    for (int s = 0; s < KSTEPS; ++s) {
+      mma16816(c0, qa[s], kr0[2 * s], kr0[2 * s + 1]);
+      mma16816(c1, qa[s], kr1[2 * s], kr1[2 * s + 1]);
+    }
+    float sc[4] = {c0[0] + c0[2], c0[1] + c0[3], c1[0] + c1[2], c1[1] + c1[3]};
+    const int tok[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
+    #pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (tok[j] >= valid) sc[j] = -INFINITY;
+    float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const float alpha = exp2f(m_run - m_new);
+    float p[4];
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) p[j] = exp2f(sc[j] - m_new);
+    l_run = l_run * alpha + (p[0] + p[1]) + (p[2] + p[3]);
+    m_run = m_new;
+    #pragma unroll
+    for (int b = 0; b < NBLK; ++b) {
+      o[b][0] *= alpha; o[b][1] *= alpha; o[b][2] *= alpha; o[b][3] *= alpha;
+    }
+    uint32_t pa[4];
+    split2(p[0], p[1], pa[0], pa[1]);
+    split2(p[2], p[3], pa[2], pa[3]);
+    #pragma unroll
+    for (int b = 0; b < NBLK; ++b) {
+      const uint32_t b0 = transpose8x8(vr0[b]);
+      const uint32_t b1 = transpose8x8(vr1[b]);
+      mma16816(o[b], pa, b0, b1);
+    }
+  }
+
+  // this warp's state for head row g (lanes of a quad share it)
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  if (g < G) {
+    #pragma unroll
+    for (int b = 0; b < NBLK; ++b) {
+      s_o[warp][g][t * DPL + 2 * b] = o[b][0] + o[b][2];
+      s_o[warp][g][t * DPL + 2 * b + 1] = o[b][1] + o[b][3];
+    }
+    if (t == 0) {
+      s_m[warp][g] = m_run;
+      s_l[warp][g] = l_run;
+    }
+  }
+  __syncthreads();
+  // merge the warps: thread handles (head, dim) pairs
+  for (int e = threadIdx.x; e < G * HD; e += kAttnWarps * 32) {
+    const int hh = e / HD, d = e % HD;
+    float M = -INFINITY;
+    #pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, s_m[w][hh]);
+    float L = 0.f, acc = 0.f;
+    #pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) {
+      const float sc = (s_m[w][hh] == -INFINITY) ? 0.f : exp2f(s_m[w][hh] - M);
+      L += sc * s_l[w][hh];
+      acc += sc * s_o[w][hh][d];
+    }
+    const int qh = h * G + hh;
+    a.part_o[((size_t)qh * kMaxSplits + split) * HD + d] = acc;
+    if (d == 0) {
+      a.part_ml[((size_t)qh * kMaxSplits + split) * 2] = M;
+      a.part_ml[((size_t)qh * kMaxSplits + split) * 2 + 1] = L;
+    }
+  }
+}
+
+template <int HD>
+__global__ void __launch_bounds__(HD) k_attn_combine(AttnArgs a) {
+  const int qh = blockIdx.x, d = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  const float* ml = a.part_ml + (size_t)qh * kMaxSplits * 2;
+  float M = -INFINITY;
+  for (int s = 0; s < a.splits; ++s) M = fmaxf(M, ml[2 * s]);
+  float L = 0.f, acc = 0.f;
+  for (int s = 0; s < a.splits; ++s) {
+    const float m = ml[2 * s];
+    const float w = (m == -INFINITY) ? 0.f : exp2f(m - M);
+    L += w * ml[2 * s + 1];
+    acc += w * a.part_o[((size_t)qh * kMaxSplits + s) * HD + d];
+  }
+  a.out[(size_t)qh * HD + d] = acc / L;
+}
+
+void attn_plan(int n_pages, int Hkv, int sms, int* splits, int* pps) {
+  const int target = 2 * sms;                   // two resident CTAs per SM (register bound)
+  int s = std::max(1, (target + Hkv - 1) / Hkv);
+  s = std::min(s, kMaxSplits);
+  s = std::min(s, std::max(1, n_pages));
+  int per = (n_pages + s - 1) / s;
+  per = std::max(per, 1);
+  *pps = per;
+  *splits = std::max(1, (n_pages + per - 1) / per);
+}
+
+template <typename K>
+static cudaError_t launch_k(K kern, dim3 grid, dim3 block, cudaStream_t st, bool pdl, const AttnArgs& a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st, bool pdl) {
+  cudaError_t e;
+  if (a.hd == 128) {
+    e = launch_k(k_attn<128>, dim3(a.splits, a.Hkv), dim3(kAttnWarps * 32), st, pdl, a);
+    if (e != cudaSuccess) return e;
+    return launch_k(k_attn_combine<128>, dim3(a.Hkv * a.G), dim3(128), st, pdl, a);
+  }
+  if (a.hd == 64) {
+    e = launch_k(k_attn<64>, dim3(a.splits, a.Hkv), dim3(kAttnWarps * 32), st, pdl, a);
+    if (e != cudaSuccess) return e;
+    return launch_k(k_attn_combine<64>, dim3(a.Hkv * a.G), dim3(64), st, pdl, a);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace bc

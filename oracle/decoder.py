@@ -96,9 +96,11 @@ def keep_count(ratio: float, n: int) -> int:
     return max(1, min(n, math.ceil(ratio * n - 1e-9)))
 
 
-def channel_select(v: np.ndarray, rp: float) -> np.ndarray:
-    """Indices of the k largest |v| (ties: lower index first), ascending."""
-    k = keep_count(rp, v.shape[0])
+def channel_select(v: np.ndarray, rp: float, k: int | None = None) -> np.ndarray:
+    """Indices of the k largest |v| (ties: lower index first), ascending;
+    k = ceil(rp*d_in - 1e-9) unless given."""
+    if k is None:
+        k = keep_count(rp, v.shape[0])
     order = np.lexsort((np.arange(v.shape[0]), -np.abs(v)))
     return np.sort(order[:k])
 

@@ -1,0 +1,131 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol,
+validates arguments on the host, and its byte account agrees with the
+oracle's (and so with the values the ByteCross README prints)."""
+import ctypes as C
+import json
+import os
+import re
+
+import pytest
+
+import activation_kv_sparsity_b200 as bc
+from oracle import byte_account as ba
+from synth import LLAMA_8B, TINY
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bytecross.h")
+GOLD = json.load(open(os.path.join(ROOT, "tests", "golden", "byte_account.json")))
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"BC_API\s+[\w\s\*]+?\b(bc_\w+)\s*\(", text)
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert len(names) >= 20
+    lib = C.CDLL(bc.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_no_undeclared_exports():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", bc.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line and line.split()[-1].startswith("bc_")}
+    assert exported == set(declared_symbols())
+
+
+def _cfg(d, max_ctx=4096):
+    return bc.config(d, max_ctx)
+
+
+def test_size_queries():
+    c = _cfg(LLAMA_8B, 131072 + 64)
+    P = (131072 + 64 + 15) // 16
+    assert bc.bc_kv_pool_bytes(C.byref(c)) == 32 * 8 * P * 2 * 16 * 128 * 2
+    assert bc.bc_meta_pool_bytes(C.byref(c)) == 32 * 8 * P * 2 * 128 * 2
+    assert 0 < bc.bc_workspace_bytes(C.byref(c)) < 256 << 20
+    bad = _cfg(dict(TINY, head_dim=96, hidden=768))
+    assert bc.bc_kv_pool_bytes(C.byref(bad)) == 0
+    assert bc.bc_workspace_bytes(C.byref(bad)) == 0
+
+
+@pytest.mark.parametrize("field,value", [("page", 32), ("head_dim", 80), ("n_kv_heads", 3), ("hidden", 500),
+                                         ("max_ctx", 0), ("rms_eps", 0.0)])
+def test_model_create_rejects_bad_config(field, value):
+    c = _cfg(TINY)
+    setattr(c, field, value)
+    w = bc.bc_weights(*([C.c_void_p(256)] * 9))
+    h = C.c_void_p()
+    st = bc.bc_model_create(C.byref(c), C.byref(w), C.c_void_p(256), C.c_void_p(256), C.c_void_p(256),
+                            1 << 30, None, C.byref(h))
+    assert st == bc.BC_EINVAL
+    assert bc.bc_last_error()
+    assert h.value is None
+
+
+def test_model_create_rejects_null_and_small_workspace():
+    c = _cfg(TINY)
+    w = bc.bc_weights(*([C.c_void_p(256)] * 9))
+    h = C.c_void_p()
+    assert bc.bc_model_create(C.byref(c), C.byref(w), None, C.c_void_p(256), C.c_void_p(256), 1 << 30, None,
+                              C.byref(h)) == bc.BC_EINVAL
+    w0 = bc.bc_weights(*([C.c_void_p(256)] * 8 + [None]))
+    assert bc.bc_model_create(C.byref(c), C.byref(w0), C.c_void_p(256), C.c_void_p(256), C.c_void_p(256), 1 << 30,
+                              None, C.byref(h)) == bc.BC_EINVAL
+    assert bc.bc_model_create(C.byref(c), C.byref(w), C.c_void_p(256), C.c_void_p(256), C.c_void_p(256), 16,
+                              None, C.byref(h)) == bc.BC_ENOMEM
+    assert bc.bc_model_create(C.byref(c), C.byref(w), C.c_void_p(260), C.c_void_p(256), C.c_void_p(256), 1 << 30,
+                              None, C.byref(h)) == bc.BC_EINVAL
+
+
+def test_single_kernel_entries_validate_on_host():
+    assert bc.bc_gemv_scratch_bytes(300) == 0
+    assert bc.bc_gemv(None, 4, 256, None, None, 4, None, None, 0, None) == bc.BC_EINVAL
+    assert bc.bc_select_topk(C.c_void_p(256), 20000, 5, C.c_void_p(256), None) == bc.BC_EINVAL
+    assert bc.bc_select_topk(C.c_void_p(256), 100, 0, C.c_void_p(256), None) == bc.BC_EINVAL
+    p = C.c_void_p(256)
+    assert bc.bc_attention(p, p, 8, 4, 96, 10, None, 1, 16, p, p, 1 << 20, None) == bc.BC_EINVAL
+
+
+MODELS = {k: dict(v, page=16) for k, v in GOLD["models"].items()}
+
+
+@pytest.mark.parametrize("case", GOLD["crossover_k"], ids=lambda c: f"{c['model']}-{c['rp']}-{c['rkv']}")
+def test_library_crossover_matches_printed(case):
+    got = bc.byte_account(MODELS[case["model"]], "both", 1024, rp=case["rp"], rkv=case["rkv"])
+    assert round(got["n_star"] / 1024, case["digits"]) == pytest.approx(case["printed"])
+    assert got["n_star"] == pytest.approx(ba.crossover(MODELS[case["model"]], case["rp"], case["rkv"]), rel=1e-6)
+
+
+def test_library_bound_and_ff_match_printed():
+    m = MODELS["llama-3.1-8b"]
+    assert round(bc.byte_account(m, "kv", 131072, rkv=0.3)["bound"], 2) == 1.60
+    assert round(bc.byte_account(m, "both", 32768, rp=0.5, rkv=0.2)["bound"], 3) == 2.172
+    assert round(bc.byte_account(m, "both", 0, rp=0.5, rkv=0.3)["n_star_ff"] / 1024, 1) == 60.0
+
+
+@pytest.mark.parametrize("mode", ["dense", "act", "kv", "both"])
+@pytest.mark.parametrize("n", [0, 15, 16, 2047, 8191, 32768, 131071])
+@pytest.mark.parametrize("cfg", [TINY, LLAMA_8B], ids=["tiny", "8b"])
+def test_library_implementation_bytes_match_oracle(cfg, mode, n):
+    kw = dict(rp=0.5, rkv=0.3, sinks=1, recent=16)
+    got = bc.byte_account(cfg, mode, n, **kw)
+    ref = ba.implementation_bytes(cfg, mode, n, **kw)
+    assert got["impl_weight_bytes"] == ref["weights"]
+    assert got["impl_head_bytes"] == ref["head"]
+    assert got["impl_kv_read_bytes"] == ref["kv_read"]
+    assert got["impl_meta_read_bytes"] == ref["meta_read"]
+    assert got["impl_kv_write_bytes"] == ref["kv_write"]
+    assert got["impl_other_bytes"] == ref["other"]
+    assert got["impl_total_bytes"] == ref["total"]
+
+
+def test_byte_account_rejects_bad_ratios():
+    c = _cfg(TINY)
+    out = bc.bc_bytes()
+    assert bc.bc_byte_account(C.byref(c), bc.BC_KV, 1.0, 0.0, 100, 1, 16, 16, C.byref(out)) == bc.BC_EINVAL
+    assert bc.bc_byte_account(C.byref(c), bc.BC_ACT, 1.5, 1.0, 100, 1, 16, 16, C.byref(out)) == bc.BC_EINVAL
+    assert bc.bc_byte_account(C.byref(c), bc.BC_KV, 1.0, 0.5, 100, 1, 0, 16, C.byref(out)) == bc.BC_EINVAL
