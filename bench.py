@@ -71,6 +71,7 @@ def barrier(ws):
 
 
 def max_over_ranks(x, ws, dev):
+    """Slowest rank's value (the job's time); one all-reduce, timing only."""
     if ws == 1:
         return x
     import torch
@@ -78,6 +79,22 @@ def max_over_ranks(x, ws, dev):
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def sum_over_ranks(x, ws, dev):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def replica_throughput(tokens_per_rank, seconds, ws, dev):
+    """Whole-job throughput of independent replicas: all ranks' tokens over
+    the slowest rank's time."""
+    return sum_over_ranks(tokens_per_rank, ws, dev) / max_over_ranks(seconds, ws, dev)
 
 
 class Clocks:
@@ -186,23 +203,49 @@ def run_ours(args, rank, ws, local):
         ms = max_over_ranks(e0.elapsed_time(e1) / steps, ws, dev)
         return ms, model.launches() - l0
 
+    def time_e2e(n):
+        # end to end through the public host-buffer entry point, at context n
+        host_logits = torch.empty(cfg["vocab"], pin_memory=True)
+        model.reset(n)
+        kwh = MODE_KW[HEAD_MODE]
+        for i in range(warm):
+            model.step_host(toks[i], HEAD_MODE, host_logits, **kwh)
+        barrier(ws)
+        t0 = time.perf_counter()
+        for i in range(steps):
+            model.step_host(toks[warm + i], HEAD_MODE, host_logits, **kwh)
+        secs = time.perf_counter() - t0
+        return {"value": round(replica_throughput(steps, secs, ws, dev), 2), "unit": "tok/s",
+                "h2d_bytes_per_step": 4, "d2h_bytes_per_step": 4 * cfg["vocab"],
+                "note": "bc_decode_step_host: token id passed by value in the launch, logits copied to "
+                        "pinned host memory, stream synchronised every step; wall clock"}
+
+    e2e = None
     cells = {}
     for n in contexts:
-        for mode in ("dense", "act", "kv", "both"):
+        if n == HEAD_CTX or (e2e is None and n == min(contexts)):
+            e2e = time_e2e(n)
+        for mode in args.modes:
             ms, launches = time_cell(mode, n)
             kw = dict(KEEP)
-            acc = bc.byte_account(cfg, mode, n, **kw)
+            # the timed steps run at contexts n+warm .. n+warm+steps-1: average their byte accounts
+            accs = [bc.byte_account(cfg, mode, n + warm + i, **kw) for i in range(steps)]
+            acc = dict(accs[0])
+            acc["impl_total_bytes"] = sum(a["impl_total_bytes"] for a in accs) / steps
             gbs = acc["impl_total_bytes"] / (ms * 1e-3) / 1e9
             cells[(mode, n)] = dict(mode=mode, context=n, ms_per_step=round(ms, 4),
                                     tok_s=round(1000.0 / ms, 2), bytes_per_step=acc["impl_total_bytes"],
                                     gbs=round(gbs, 1), frac_of_measured_peak=round(gbs / peak, 4),
                                     paper_bound=round(acc["bound"], 4), launches_per_step=launches // steps)
     for n in contexts:
+        if ("dense", n) not in cells:
+            continue
         d = cells[("dense", n)]["ms_per_step"]
         for mode in ("act", "kv", "both"):
-            cells[(mode, n)]["speedup_vs_dense"] = round(d / cells[(mode, n)]["ms_per_step"], 4)
+            if (mode, n) in cells:
+                cells[(mode, n)]["speedup_vs_dense"] = round(d / cells[(mode, n)]["ms_per_step"], 4)
 
-    head = cells.get((HEAD_MODE, HEAD_CTX)) or cells[(HEAD_MODE, contexts[0])]
+    head = cells.get((HEAD_MODE, HEAD_CTX)) or cells.get((HEAD_MODE, contexts[0])) or next(iter(cells.values()))
     head_ctx = head["context"]
     head_launches = head["launches_per_step"] * steps
 
@@ -236,21 +279,6 @@ def run_ours(args, rank, ws, local):
     # point over 8 layers' pages
     attn = None
 
-    # end to end through the public host-buffer entry point
-    host_logits = torch.empty(cfg["vocab"], pin_memory=True)
-    model.reset(head_ctx)
-    kwh = MODE_KW[HEAD_MODE]
-    for i in range(warm):
-        model.step_host(toks[i], HEAD_MODE, host_logits, **kwh)
-    barrier(ws)
-    t0 = time.perf_counter()
-    for i in range(steps):
-        model.step_host(toks[warm + i], HEAD_MODE, host_logits, **kwh)
-    e2e_s = max_over_ranks(time.perf_counter() - t0, ws, dev)
-    e2e = {"value": round(ws * steps / e2e_s, 2), "unit": "tok/s", "h2d_bytes_per_step": 4,
-           "d2h_bytes_per_step": 4 * cfg["vocab"],
-           "note": "bc_decode_step_host: token id passed by value in the launch, logits copied to pinned host memory, stream synchronised every step"}
-
     clk = clocks.summary()
     # measured crossings against the byte-account n*
     crossings = {}
@@ -261,7 +289,7 @@ def run_ours(args, rank, ws, local):
 
     result = {
         "metric": METRIC,
-        "value": round(ws * 1000.0 / head["ms_per_step"], 2),
+        "value": round(replica_throughput(steps, head["ms_per_step"] * steps / 1000.0, ws, dev), 2),
         "unit": "tok/s",
         "n_gpus": ws,
         "steps": steps,
@@ -300,6 +328,8 @@ def measured_crossing(cells, contexts):
     interpolated linearly between the sampled contexts (the README's
     convention for latency crossings)."""
     ctx = sorted(contexts)
+    if not all(("act", n) in cells and ("kv", n) in cells for n in ctx):
+        return {"act_vs_kv_tokens": None}
     diff = [(n, cells[("act", n)]["ms_per_step"] - cells[("kv", n)]["ms_per_step"]) for n in ctx]
     for (n0, d0), (n1, d1) in zip(diff, diff[1:]):
         if d0 < 0 <= d1:
@@ -429,6 +459,59 @@ def run_reference(args, rank, ws, local):
     }
 
 
+def run_kernel_only(args, local):
+    """Times one kernel alone on a small case (for profiler captures): the
+    gathered gate/up GEMV of one layer (235 MB dense, 117 MB at rp 0.5) or
+    the dense split-K attention of one layer at 128K context (537 MB)."""
+    import torch
+    import activation_kv_sparsity_b200 as bc
+    from synth import LLAMA_8B
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = LLAMA_8B
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    stream = torch.cuda.current_stream(dev)
+    if args.only_kernel == "gemv_gateup":
+        d, d_out = cfg["hidden"], 2 * cfg["intermediate"]
+        W = (torch.randn(d, d_out, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        k = math.ceil(0.5 * d - 1e-9)
+        idx = torch.sort(torch.randperm(d, device=dev, generator=g)[:k])[0].to(torch.int32)
+        x = torch.randn(d, generator=g, device=dev)
+        y = torch.empty(d_out, device=dev)
+        scratch = torch.zeros(bc.bc_gemv_scratch_bytes(d_out), dtype=torch.uint8, device=dev)
+        nbytes = k * d_out * 2 + k * 8
+
+        def launch():
+            bc.gemv(W, x, idx, y, scratch, stream)
+    else:
+        Hkv, G, hd, n_tok = cfg["n_kv_heads"], cfg["n_heads"] // cfg["n_kv_heads"], cfg["head_dim"], 131073
+        P = -(-n_tok // 16)
+        pool = torch.randn(Hkv, P, 2, 16, hd, generator=g, device=dev).to(torch.bfloat16)
+        q = torch.randn(Hkv * G, hd, generator=g, device=dev)
+        out = torch.empty(Hkv * G, hd, device=dev)
+        scratch = torch.zeros(bc.bc_attention_scratch_bytes(Hkv * G, hd), dtype=torch.uint8, device=dev)
+        nbytes = Hkv * n_tok * 2 * hd * 2
+
+        def launch():
+            bc.attention(q, pool, Hkv, G, hd, P, None, P, n_tok, out, scratch, stream)
+    for _ in range(args.warmup):
+        launch()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        launch()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    peak, kind = peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"kernel": args.only_kernel, "ms_per_launch": round(ms, 5), "algorithmic_bytes": nbytes,
+            "gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "peak": peak, "peak_kind": kind,
+            "note": "includes the combine kernel" if args.only_kernel == "attention" else ""}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -437,13 +520,22 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--contexts", type=int, nargs="+", default=list(CONTEXTS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--modes", nargs="+", default=["dense", "act", "kv", "both"],
+                    choices=["dense", "act", "kv", "both"])
+    ap.add_argument("--only-kernel", choices=("gemv_gateup", "attention"),
+                    help="time one kernel alone on a small case (profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    rank, ws, local = dist_init(args.gpus)
     if args.impl == "reference":
-        if rank == 0:
-            print(json.dumps(run_reference(args, rank, ws, local)))
+        # the oracle arm runs on rank 0 alone; other ranks exit without work
+        if int(os.environ.get("RANK", "0")) == 0:
+            print(json.dumps(run_reference(args, 0, int(os.environ.get("WORLD_SIZE", "1")),
+                                           int(os.environ.get("LOCAL_RANK", "0")))))
+        return
+    rank, ws, local = dist_init(args.gpus)
+    if args.only_kernel:
+        print(json.dumps(run_kernel_only(args, local)))
         return
     res = run_ours(args, rank, ws, local)
     if rank == 0:
