@@ -63,6 +63,8 @@ _SIGS = {
     "bc_trace": (C.c_int, [_P, C.c_int, C.c_int, C.POINTER(_P), C.POINTER(C.c_int), C.POINTER(C.c_int)]),
     "bc_gemv_scratch_bytes": (C.c_size_t, [C.c_int]),
     "bc_gemv": (C.c_int, [_P, C.c_int, C.c_int, _P, _P, C.c_int, _P, _P, C.c_size_t, _P]),
+    "bc_gemv_noalloc_max_dout": (C.c_int, []),
+    "bc_gemv_noalloc": (C.c_int, [_P, C.c_int, C.c_int, _P, _P, C.c_int, _P, _P]),
     "bc_select_topk": (C.c_int, [_P, C.c_int, C.c_int, _P, _P]),
     "bc_attention_scratch_bytes": (C.c_size_t, [C.c_int, C.c_int]),
     "bc_attention": (C.c_int, [_P, _P, C.c_int, C.c_int, C.c_int, C.c_int, _P, C.c_int, C.c_int, _P, _P,
@@ -195,6 +197,15 @@ def gemv(W, x, idx, y, scratch, stream=None):
                   C.c_void_p(idx.data_ptr()) if idx is not None else None, k, C.c_void_p(y.data_ptr()),
                   C.c_void_p(scratch.data_ptr()), scratch.numel() * scratch.element_size(),
                   _stream_ptr(stream)), "bc_gemv")
+
+
+def gemv_noalloc(W, x, idx, y, stream=None):
+    """bc_gemv without a scratch argument (scratch is a static device array)."""
+    d_in, d_out = W.shape
+    k = d_in if idx is None else idx.numel()
+    check(bc_gemv_noalloc(C.c_void_p(W.data_ptr()), d_in, d_out, C.c_void_p(x.data_ptr()),
+                          C.c_void_p(idx.data_ptr()) if idx is not None else None, k, C.c_void_p(y.data_ptr()),
+                          _stream_ptr(stream)), "bc_gemv_noalloc")
 
 
 def select_topk(v, k, idx, stream=None):

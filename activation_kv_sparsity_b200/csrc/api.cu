@@ -39,6 +39,8 @@ static bc_status cuda_fail(cudaError_t e, const char* where) {
 
 extern "C" const char* bc_last_error(void) { return g_err.c_str(); }
 
+void bc::set_error(const char* msg) { g_err = msg; }
+
 extern "C" const char* bc_status_string(bc_status s) {
   switch (s) {
     case BC_OK: return "ok";

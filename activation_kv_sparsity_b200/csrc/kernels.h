@@ -7,6 +7,9 @@
 
 namespace bc {
 
+// Records the message bc_last_error() returns on this thread.
+void set_error(const char* msg);
+
 // ------------------------------------------------------------------ GEMV
 enum GemvEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_QKV = 2 };
 

@@ -212,6 +212,24 @@ BC_API size_t bc_gemv_scratch_bytes(int d_out);
 BC_API bc_status bc_gemv(const void* W, int d_in, int d_out, const float* x, const int* idx, int k,
                          float* y, void* scratch, size_t scratch_bytes, void* stream);
 
+/* Column-gathered GEMV that allocates nothing: the same computation and
+ * arguments as bc_gemv without the scratch buffer.  The paper has no
+ * counterpart; this is for callers that cannot allocate device memory, such
+ * as an operator inside another framework whose allocator owns the device
+ * memory and hands the operator only its inputs and outputs, or a serving
+ * path that must not call cudaMalloc (it can synchronise the device).
+ * The split-K scratch lives in a file-scope __device__ array of
+ * 8 MiB + 512 B, held on every GPU that loads the library until exit; d_out
+ * above bc_gemv_noalloc_max_dout() (32768) is rejected with BC_EINVAL.  The
+ * first call on a device, with that device current, looks the array's
+ * address up; make it before any stream capture.  Every call clears the
+ * tickets it needs and shares the array with every other call: calls that
+ * overlap on the GPU race and must be serialised by the caller.  Allocates
+ * no device memory (no cudaMalloc, cudaFree or allocating library call). */
+BC_API int bc_gemv_noalloc_max_dout(void);
+BC_API bc_status bc_gemv_noalloc(const void* W, int d_in, int d_out, const float* x, const int* idx, int k,
+                                 float* y, void* stream);
+
 /* Exact top-k selection: writes to idx (device int32 [k]) the k indices of
  * largest |v| (v: device f32 [n]), ascending; ties go to the lower index.
  * 1 <= k <= n <= 16384. */
