@@ -85,6 +85,12 @@ struct Layout {
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Ticket counters: 4 GEMV sites x column tiles, then attention and page
+// select per kv head.  Zeroed at create; every kernel leaves its own at zero.
+static size_t counter_bytes(const bc_config* c, const Layout& y) {
+  return 4 * (4 * (size_t)(y.max_dout / 128) + 2 * (size_t)c->n_kv_heads);
+}
+
 static Layout make_layout(const bc_config* c) {
   Layout y;
   const size_t L = c->n_layers, d = c->hidden, f = c->intermediate;
@@ -113,8 +119,8 @@ static Layout make_layout(const bc_config* c) {
   y.pages = take(4 * L * c->n_kv_heads * (size_t)y.Pmax);
   y.part_o = take(4 * (size_t)c->n_heads * kMaxSplits * c->head_dim);
   y.part_ml = take(4 * (size_t)c->n_heads * kMaxSplits * 2);
-  y.gemv_part = take(4 * (size_t)kGemvMaxChunks * y.max_dout);
-  y.counters = take(4 * 4 * (size_t)(y.max_dout / kColTile));
+  y.gemv_part = take(4 * (size_t)kGemvMaxContrib * y.max_dout);
+  y.counters = take(counter_bytes(c, y));
   y.total = o;
   return y;
 }
@@ -155,6 +161,7 @@ struct bc_model {
   // what the last step left in the traces
   int last_k[4];       // kept channels per site (0 = no selection)
   int last_P, last_K;  // pages after the append, kept pages (0 = no selection)
+  bool last_act;       // the last step ranked activations (XN, XN2, H traces valid)
 };
 
 template <typename T>
@@ -197,7 +204,8 @@ extern "C" bc_status bc_model_create(const bc_config* cfg, const bc_weights* w, 
   m->launches = 0;
   memset(m->last_k, 0, sizeof m->last_k);
   m->last_P = m->last_K = 0;
-  cudaError_t e = cudaMemsetAsync(m->ws + lay.counters, 0, 4 * 4 * (size_t)(lay.max_dout / kColTile), m->stream);
+  m->last_act = false;
+  cudaError_t e = cudaMemsetAsync(m->ws + lay.counters, 0, counter_bytes(cfg, lay), m->stream);
   if (e != cudaSuccess) {
     delete m;
     return cuda_fail(e, "bc_model_create: clearing counters");
@@ -269,42 +277,51 @@ static bc_status check_step(const bc_model* m, bc_mode mode, float rp, float rkv
   return BC_OK;
 }
 
-static cudaError_t step_select(bc_model* m, int prep, int n, bool sel, int k, const float* v,
-                               const __nv_bfloat16* gain, const __nv_bfloat16* emb, float* x_out,
-                               float* out, int* idx) {
+static cudaError_t step_select(bc_model* m, int prep, int n, int k, const float* x,
+                               const __nv_bfloat16* gain, const __nv_bfloat16* emb, float* x_init,
+                               float* vout, int* idx) {
   SelectArgs s;
   s.prep = prep;
   s.n = n;
   s.k = k;
-  s.do_select = sel ? 1 : 0;
-  s.v = v;
+  s.x = x;
   s.gain = gain;
-  s.eps = m->cfg.rms_eps;
   s.embed_row = emb;
-  s.x_out = x_out;
-  s.out = out;
+  s.x_init = x_init;
+  s.vout = vout;
   s.idx = idx;
   return launch_select(s, m->stream, true);
 }
 
-static cudaError_t step_gemv(bc_model* m, int site, const __nv_bfloat16* W, int d_in, int d_out,
-                             const float* x, const int* idx, int k, int epi, float* y,
-                             float* y_copy, const QkvEpilogue* qe) {
+static unsigned* gemv_counters(bc_model* m, int site) {
+  return at<unsigned>(m, m->lay.counters) + site * (m->lay.max_dout / 128);
+}
+
+static cudaError_t step_gemv(bc_model* m, int site, const __nv_bfloat16* W, int d_in, int d_out, int prep,
+                             const float* x, const __nv_bfloat16* gain, const __nv_bfloat16* emb,
+                             float* x_init, const int* idx, int k, int epi, float* y, float* y_copy,
+                             const QkvEpilogue* qe) {
   GemvArgs g;
+  memset(&g, 0, sizeof g);
   g.W = W;
   g.d_in = d_in;
   g.d_out = d_out;
+  g.prep = prep;
   g.x = x;
+  g.gain = gain;
+  g.eps = m->cfg.rms_eps;
+  g.embed_row = emb;
+  g.x_init = x_init;
   g.idx = idx;
   g.k = k;
-  gemv_plan(k, d_out, m->sms, kGemvMaxChunks, &g.chunk, &g.n_chunks);
+  gemv_plan(k, d_out, m->sms, &g.TW, &g.S, &g.C);
+  g.max_rows = (k + g.S * g.C - 1) / (g.S * g.C);
   g.partial = at<float>(m, m->lay.gemv_part);
-  g.counters = at<unsigned>(m, m->lay.counters) + site * (m->lay.max_dout / kColTile);
+  g.counters = gemv_counters(m, site);
   g.epi = epi;
   g.y = y;
   g.y_copy = y_copy;
   if (qe) g.qkv = *qe;
-  else memset(&g.qkv, 0, sizeof g.qkv);
   return launch_gemv(g, m->stream, true);
 }
 
@@ -341,9 +358,12 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
   float* x = at<float>(m, y.x);
   const size_t kv_layer = (size_t)Hkv * Pmax * 2 * kPage * hd;
   const size_t meta_layer = (size_t)Hkv * Pmax * 2 * hd;
+  unsigned* att_counters = gemv_counters(m, 4);
+  unsigned* page_counters = att_counters + Hkv;
 
   int splits, pps;
   attn_plan(K, Hkv, m->sms, &splits, &pps);
+  long long launches = 0;
 
   for (int l = 0; l < L; ++l) {
     float* xn = at<float>(m, y.xn) + (size_t)l * d;
@@ -362,10 +382,18 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
     int* pages = at<int>(m, y.pages) + (size_t)l * Hkv * Pmax;
     __nv_bfloat16* kvl = m->kv + l * kv_layer;
     __nv_bfloat16* metal = m->meta + l * meta_layer;
+    const __nv_bfloat16* g_attn = attn_norm + (size_t)l * d;
+    const __nv_bfloat16* g_mlp = mlp_norm + (size_t)l * d;
+    const bool first = l == 0;
 
-    // attention block
-    BC_CUDA(step_select(m, l == 0 ? PREP_EMBED_NORM : PREP_NORM, d, act, k_qkv, x,
-                        attn_norm + (size_t)l * d, emb, x, xn, s_qkv), "select qkv");
+    // attention block: [select] -> q/k/v GEMV (RMSNorm folded in; rotary,
+    // append and page bounds in the epilogue) -> [page scores + select] ->
+    // split-K attention with fused combine
+    if (act) {
+      BC_CUDA(step_select(m, first ? SP_EMBED_NORM : SP_NORM, d, k_qkv, x, g_attn, emb, x, xn, s_qkv),
+              "select qkv");
+      ++launches;
+    }
     QkvEpilogue qe;
     qe.Hq = Hq;
     qe.Hkv = Hkv;
@@ -376,13 +404,13 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
     qe.q_out = q;
     qe.kv_layer = kvl;
     qe.meta_layer = metal;
-    BC_CUDA(step_gemv(m, 0, wqkv + (size_t)l * d * nqkv, d, nqkv, xn, act ? s_qkv : nullptr, k_qkv,
-                      EPI_QKV, qkv, nullptr, &qe), "gemv qkv");
+    BC_CUDA(step_gemv(m, 0, wqkv + (size_t)l * d * nqkv, d, nqkv, first ? GP_EMBED_NORM : GP_NORM, x, g_attn,
+                      emb, x, act ? s_qkv : nullptr, k_qkv, EPI_QKV, qkv, nullptr, &qe), "gemv qkv");
+    ++launches;
     if (kvs) {
-      PageScoreArgs ps{q, metal, Hkv, G, hd, Pmax, P, pscore};
-      BC_CUDA(launch_page_scores(ps, m->stream, true), "page scores");
-      PageSelectArgs pl{pscore, Hkv, Pmax, P, K, sinks, recent, pages};
-      BC_CUDA(launch_page_select(pl, m->stream, true), "page select");
+      PageArgs pa{q, metal, Hkv, G, hd, Pmax, P, K, sinks, recent, pscore, pages, page_counters};
+      BC_CUDA(launch_pages(pa, m->stream, true), "page scores and select");
+      ++launches;
     }
     AttnArgs aa;
     aa.q = q;
@@ -398,39 +426,46 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
     aa.pages_per_split = pps;
     aa.part_o = at<float>(m, y.part_o);
     aa.part_ml = at<float>(m, y.part_ml);
+    aa.counters = att_counters;
     aa.out = attn;
     BC_CUDA(launch_attention(aa, m->stream, true), "attention");
-    if (act)
-      BC_CUDA(step_select(m, PREP_NONE, hq, true, k_o, attn, nullptr, nullptr, nullptr, nullptr, s_o),
-              "select o");
-    BC_CUDA(step_gemv(m, 1, wo + (size_t)l * hq * d, hq, d, attn, act ? s_o : nullptr, k_o, EPI_RESID,
-                      x, nullptr, nullptr), "gemv o");
-    // feed-forward block
-    BC_CUDA(step_select(m, PREP_NORM, d, act, k_gu, x, mlp_norm + (size_t)l * d, nullptr, nullptr,
-                        xn2, s_gu), "select gate/up");
-    BC_CUDA(step_gemv(m, 2, wgu + (size_t)l * d * 2 * f, d, 2 * f, xn2, act ? s_gu : nullptr, k_gu,
-                      EPI_STORE, gu, nullptr, nullptr), "gemv gate/up");
-    BC_CUDA(step_select(m, PREP_SWIGLU, f, act, k_d, gu, nullptr, nullptr, nullptr, hmid, s_d),
-            "select down");
-    BC_CUDA(step_gemv(m, 3, wd + (size_t)l * f * d, f, d, hmid, act ? s_d : nullptr, k_d, EPI_RESID,
-                      x, xo, nullptr), "gemv down");
+    ++launches;
+    if (act) {
+      BC_CUDA(step_select(m, SP_NONE, hq, k_o, attn, nullptr, nullptr, nullptr, nullptr, s_o), "select o");
+      ++launches;
+    }
+    BC_CUDA(step_gemv(m, 1, wo + (size_t)l * hq * d, hq, d, GP_NONE, attn, nullptr, nullptr, nullptr,
+                      act ? s_o : nullptr, k_o, EPI_RESID, x, nullptr, nullptr), "gemv o");
+    ++launches;
+    // feed-forward block: [select] -> gate/up GEMV (RMSNorm folded in) ->
+    // [select] -> down GEMV (SwiGLU folded in) + residual
+    if (act) {
+      BC_CUDA(step_select(m, SP_NORM, d, k_gu, x, g_mlp, nullptr, nullptr, xn2, s_gu), "select gate/up");
+      ++launches;
+    }
+    BC_CUDA(step_gemv(m, 2, wgu + (size_t)l * d * 2 * f, d, 2 * f, GP_NORM, x, g_mlp, nullptr, nullptr,
+                      act ? s_gu : nullptr, k_gu, EPI_STORE, gu, nullptr, nullptr), "gemv gate/up");
+    ++launches;
+    if (act) {
+      BC_CUDA(step_select(m, SP_SWIGLU, f, k_d, gu, nullptr, nullptr, nullptr, hmid, s_d), "select down");
+      ++launches;
+    }
+    BC_CUDA(step_gemv(m, 3, wd + (size_t)l * f * d, f, d, GP_SWIGLU, gu, nullptr, nullptr, nullptr,
+                      act ? s_d : nullptr, k_d, EPI_RESID, x, xo, nullptr), "gemv down");
+    ++launches;
   }
-  float* xf = at<float>(m, y.xf);
-  BC_CUDA(step_select(m, PREP_NORM, d, false, d, x, static_cast<const __nv_bfloat16*>(m->w.final_norm),
-                      nullptr, nullptr, xf, nullptr), "final norm");
-  LmHeadArgs lm{static_cast<const __nv_bfloat16*>(m->w.lm_head), c.vocab, d, xf, logits};
+  LmHeadArgs lm{static_cast<const __nv_bfloat16*>(m->w.lm_head), c.vocab, d, x,
+                static_cast<const __nv_bfloat16*>(m->w.final_norm), c.rms_eps, logits};
   BC_CUDA(launch_lmhead(lm, m->sms, m->stream, true), "lm head");
+  ++launches;
 
-  // launches: per layer norm/select, q/k/v, attention + combine, o, norm/select,
-  // gate/up, swiglu/select, down; the kv branch adds scores and page select,
-  // the projection branch the select of the attention output; then the
-  // final norm and the LM head
-  m->launches += (long long)L * (9 + (kvs ? 2 : 0) + (act ? 1 : 0)) + 2;
+  m->launches += launches;
   m->n = n_tok;
   m->last_k[0] = act ? k_qkv : 0;
   m->last_k[1] = act ? k_o : 0;
   m->last_k[2] = act ? k_gu : 0;
   m->last_k[3] = act ? k_d : 0;
+  m->last_act = act;
   m->last_P = P;
   m->last_K = kvs ? K : 0;
   return BC_OK;
@@ -470,14 +505,14 @@ extern "C" bc_status bc_trace(const bc_model* m, int layer, bc_trace_kind kind, 
   size_t off = 0;
   int n = 0, st = 0;
   switch (kind) {
-    case BC_TRACE_XN: off = y.xn + 4ull * layer * d; n = d; break;
+    case BC_TRACE_XN: off = y.xn + 4ull * layer * d; n = m->last_act ? d : 0; break;
     case BC_TRACE_SEL_QKV: off = y.sel_qkv + 4ull * layer * d; n = m->last_k[0]; break;
     case BC_TRACE_Q: off = y.q + 4ull * layer * hq; n = hq; break;
     case BC_TRACE_ATTN: off = y.attn + 4ull * layer * hq; n = hq; break;
     case BC_TRACE_SEL_O: off = y.sel_o + 4ull * layer * hq; n = m->last_k[1]; break;
-    case BC_TRACE_XN2: off = y.xn2 + 4ull * layer * d; n = d; break;
+    case BC_TRACE_XN2: off = y.xn2 + 4ull * layer * d; n = m->last_act ? d : 0; break;
     case BC_TRACE_SEL_GU: off = y.sel_gu + 4ull * layer * d; n = m->last_k[2]; break;
-    case BC_TRACE_H: off = y.h + 4ull * layer * f; n = f; break;
+    case BC_TRACE_H: off = y.h + 4ull * layer * f; n = m->last_act ? f : 0; break;
     case BC_TRACE_SEL_D: off = y.sel_d + 4ull * layer * f; n = m->last_k[3]; break;
     case BC_TRACE_X: off = y.xo + 4ull * layer * d; n = d; break;
     case BC_TRACE_PAGE_SCORES:
@@ -496,7 +531,7 @@ extern "C" bc_status bc_trace(const bc_model* m, int layer, bc_trace_kind kind, 
 // ------------------------------------------------------------------ single kernels
 extern "C" size_t bc_gemv_scratch_bytes(int d_out) {
   if (d_out <= 0 || d_out % kColTile) return 0;
-  return align256(4ull * kGemvMaxChunks * d_out) + align256(4ull * (d_out / kColTile));
+  return align256(4ull * kGemvMaxContrib * d_out) + align256(4ull * (d_out / 128));
 }
 
 extern "C" bc_status bc_gemv(const void* W, int d_in, int d_out, const float* x, const int* idx, int k,
@@ -506,19 +541,20 @@ extern "C" bc_status bc_gemv(const void* W, int d_in, int d_out, const float* x,
   if (k < 1 || k > d_in || (!idx && k != d_in)) return fail(BC_EINVAL, "k must be in [1, d_in] (= d_in without idx)");
   if (scratch_bytes < bc_gemv_scratch_bytes(d_out)) return fail(BC_ENOMEM, "scratch too small");
   GemvArgs g;
+  memset(&g, 0, sizeof g);
   g.W = static_cast<const __nv_bfloat16*>(W);
   g.d_in = d_in;
   g.d_out = d_out;
+  g.prep = GP_NONE;
   g.x = x;
   g.idx = idx;
   g.k = k;
-  gemv_plan(k, d_out, device_sms(), kGemvMaxChunks, &g.chunk, &g.n_chunks);
+  gemv_plan(k, d_out, device_sms(), &g.TW, &g.S, &g.C);
+  g.max_rows = (k + g.S * g.C - 1) / (g.S * g.C);
   g.partial = static_cast<float*>(scratch);
-  g.counters = reinterpret_cast<unsigned*>(static_cast<char*>(scratch) + align256(4ull * kGemvMaxChunks * d_out));
+  g.counters = reinterpret_cast<unsigned*>(static_cast<char*>(scratch) + align256(4ull * kGemvMaxContrib * d_out));
   g.epi = EPI_STORE;
   g.y = y;
-  g.y_copy = nullptr;
-  memset(&g.qkv, 0, sizeof g.qkv);
   BC_CUDA(launch_gemv(g, static_cast<cudaStream_t>(stream), true), "bc_gemv");
   return BC_OK;
 }
@@ -528,11 +564,10 @@ extern "C" bc_status bc_select_topk(const float* v, int n, int k, int* idx, void
   if (n < 1 || n > kMaxSelect || k < 1 || k > n) return fail(BC_EINVAL, "need 1 <= k <= n <= 16384");
   SelectArgs s;
   memset(&s, 0, sizeof s);
-  s.prep = PREP_NONE;
+  s.prep = SP_NONE;
   s.n = n;
   s.k = k;
-  s.do_select = 1;
-  s.v = v;
+  s.x = v;
   s.idx = idx;
   BC_CUDA(launch_select(s, static_cast<cudaStream_t>(stream), true), "bc_select_topk");
   return BC_OK;
@@ -540,7 +575,8 @@ extern "C" bc_status bc_select_topk(const float* v, int n, int k, int* idx, void
 
 extern "C" size_t bc_attention_scratch_bytes(int n_q_heads, int head_dim) {
   if (n_q_heads <= 0 || head_dim <= 0) return 0;
-  return align256(4ull * n_q_heads * kMaxSplits * head_dim) + align256(4ull * n_q_heads * kMaxSplits * 2);
+  return align256(4ull * n_q_heads * kMaxSplits * head_dim) + align256(4ull * n_q_heads * kMaxSplits * 2) +
+         align256(4ull * n_q_heads);
 }
 
 extern "C" bc_status bc_attention(const float* q, const void* kv, int n_kv_heads, int group, int head_dim,
@@ -552,7 +588,8 @@ extern "C" bc_status bc_attention(const float* q, const void* kv, int n_kv_heads
   if (n_tok < 1 || n_pages < 1 || Pmax < n_pages || (n_tok + kPage - 1) / kPage > Pmax)
     return fail(BC_EINVAL, "bad page counts");
   if (!pages && n_pages != (n_tok + kPage - 1) / kPage) return fail(BC_EINVAL, "without a page list n_pages must cover n_tok");
-  if (scratch_bytes < bc_attention_scratch_bytes(n_kv_heads * group, head_dim)) return fail(BC_ENOMEM, "scratch too small");
+  const int nq = n_kv_heads * group;
+  if (scratch_bytes < bc_attention_scratch_bytes(nq, head_dim)) return fail(BC_ENOMEM, "scratch too small");
   AttnArgs a;
   a.q = q;
   a.kv = static_cast<const __nv_bfloat16*>(kv);
@@ -564,8 +601,12 @@ extern "C" bc_status bc_attention(const float* q, const void* kv, int n_kv_heads
   a.n_pages = n_pages;
   a.n_tok = n_tok;
   attn_plan(n_pages, n_kv_heads, device_sms(), &a.splits, &a.pages_per_split);
-  a.part_o = static_cast<float*>(scratch);
-  a.part_ml = reinterpret_cast<float*>(static_cast<char*>(scratch) + align256(4ull * n_kv_heads * group * kMaxSplits * head_dim));
+  char* sc = static_cast<char*>(scratch);
+  const size_t o_bytes = align256(4ull * nq * kMaxSplits * head_dim);
+  const size_t ml_bytes = align256(4ull * nq * kMaxSplits * 2);
+  a.part_o = reinterpret_cast<float*>(sc);
+  a.part_ml = reinterpret_cast<float*>(sc + o_bytes);
+  a.counters = reinterpret_cast<unsigned*>(sc + o_bytes + ml_bytes);
   a.out = out;
   BC_CUDA(launch_attention(a, static_cast<cudaStream_t>(stream), true), "bc_attention");
   return BC_OK;

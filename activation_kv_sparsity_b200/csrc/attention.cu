@@ -19,8 +19,9 @@
 // Value fragments are transposed in registers with movmatrix.  Each lane
 // ends with its head row's output over hd/4 consecutive dims.
 //
-// Partials (m, l, o) per (query head, split) use base-2 logits; the combine
-// kernel merges them: o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+// Partials (m, l, o) per (query head, split) use base-2 logits.  The last
+// CTA of each kv head to finish (an atomic ticket, no spinning) merges them:
+// o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, summing in split order.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -203,31 +204,83 @@ __global__ void __launch_bounds__(kAttnWarps * 32) k_attn(AttnArgs a) {
       a.part_ml[((size_t)qh * kMaxSplits + split) * 2 + 1] = L;
     }
   }
-}
 
-template <int HD>
-__global__ void __launch_bounds__(HD) k_attn_combine(AttnArgs a) {
-  const int qh = blockIdx.x, d = threadIdx.x;
-  pdl_wait();
-  pdl_trigger();
-  const float* ml = a.part_ml + (size_t)qh * kMaxSplits * 2;
-  float M = -INFINITY;
-  for (int s = 0; s < a.splits; ++s) M = fmaxf(M, ml[2 * s]);
-  float L = 0.f, acc = 0.f;
-  for (int s = 0; s < a.splits; ++s) {
-    const float m = ml[2 * s];
-    const float w = (m == -INFINITY) ? 0.f : exp2f(m - M);
-    L += w * ml[2 * s + 1];
-    acc += w * a.part_o[((size_t)qh * kMaxSplits + s) * HD + d];
+  // the last split of this kv head to finish merges the partials
+  __shared__ int s_last;
+  __shared__ float s_w[8][kMaxSplits];
+  __shared__ float s_inv[8];
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&a.counters[h], 1u) == (unsigned)(a.splits - 1));
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (threadIdx.x == 0) a.counters[h] = 0u;
+  __shared__ float s_l2[8][kMaxSplits];
+  #pragma unroll 4
+  for (int e = threadIdx.x; e < G * kMaxSplits; e += kAttnWarps * 32) {
+    const int hh = e / kMaxSplits, sp = e % kMaxSplits;
+    float m = -INFINITY, l = 0.f;
+    if (sp < a.splits) {
+      const float2 ml = *reinterpret_cast<const float2*>(&a.part_ml[((size_t)(h * G + hh) * kMaxSplits + sp) * 2]);
+      m = ml.x;
+      l = ml.y;
+    }
+    s_w[hh][sp] = m;
+    s_l2[hh][sp] = l;
   }
-  a.out[(size_t)qh * HD + d] = acc / L;
+  __syncthreads();
+  // one warp per head: max, weights and normaliser over the splits
+  for (int hh = threadIdx.x >> 5; hh < G; hh += kAttnWarps) {
+    const int ln = threadIdx.x & 31;
+    float M = -INFINITY;
+    for (int sp = ln; sp < a.splits; sp += 32) M = fmaxf(M, s_w[hh][sp]);
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    for (int sp = ln; sp < kMaxSplits; sp += 32) {
+      const float m = s_w[hh][sp];
+      const float w = (sp < a.splits && m != -INFINITY) ? exp2f(m - M) : 0.f;
+      s_w[hh][sp] = w;
+      L += w * s_l2[hh][sp];
+    }
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (ln == 0) s_inv[hh] = 1.0f / L;
+  }
+  __syncthreads();
+  // each thread owns 4 consecutive outputs (a float4) and sums the splits in
+  // order, 8 split loads in flight at a time
+  for (int e4 = threadIdx.x; e4 < G * HD / 4; e4 += kAttnWarps * 32) {
+    const int hh = (e4 * 4) / HD, d = (e4 * 4) % HD;
+    const float4* po = reinterpret_cast<const float4*>(a.part_o + (size_t)(h * G + hh) * kMaxSplits * HD + d);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp0 = 0; sp0 < a.splits; sp0 += 8) {
+      float4 v[8];
+      #pragma unroll
+      for (int u = 0; u < 8; ++u)
+        v[u] = sp0 + u < a.splits ? __ldcg(po + (size_t)(sp0 + u) * (HD / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      #pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float w = sp0 + u < a.splits ? s_w[hh][sp0 + u] : 0.f;
+        acc.x += w * v[u].x;
+        acc.y += w * v[u].y;
+        acc.z += w * v[u].z;
+        acc.w += w * v[u].w;
+      }
+    }
+    const float inv = s_inv[hh];
+    *reinterpret_cast<float4*>(a.out + (size_t)(h * G + hh) * HD + d) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
 }
 
 void attn_plan(int n_pages, int Hkv, int sms, int* splits, int* pps) {
   const int target = 2 * sms;                   // two resident CTAs per SM (register bound)
   int s = std::max(1, (target + Hkv - 1) / Hkv);
   s = std::min(s, kMaxSplits);
-  s = std::min(s, std::max(1, n_pages));
+  // at least two pages per warp: short lists use fewer, fuller splits
+  s = std::min(s, std::max(1, n_pages / (2 * kAttnWarps)));
   int per = (n_pages + s - 1) / s;
   per = std::max(per, 1);
   *pps = per;
@@ -249,17 +302,8 @@ static cudaError_t launch_k(K kern, dim3 grid, dim3 block, cudaStream_t st, bool
 }
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st, bool pdl) {
-  cudaError_t e;
-  if (a.hd == 128) {
-    e = launch_k(k_attn<128>, dim3(a.splits, a.Hkv), dim3(kAttnWarps * 32), st, pdl, a);
-    if (e != cudaSuccess) return e;
-    return launch_k(k_attn_combine<128>, dim3(a.Hkv * a.G), dim3(128), st, pdl, a);
-  }
-  if (a.hd == 64) {
-    e = launch_k(k_attn<64>, dim3(a.splits, a.Hkv), dim3(kAttnWarps * 32), st, pdl, a);
-    if (e != cudaSuccess) return e;
-    return launch_k(k_attn_combine<64>, dim3(a.Hkv * a.G), dim3(64), st, pdl, a);
-  }
+  if (a.hd == 128) return launch_k(k_attn<128>, dim3(a.splits, a.Hkv), dim3(kAttnWarps * 32), st, pdl, a);
+  if (a.hd == 64) return launch_k(k_attn<64>, dim3(a.splits, a.Hkv), dim3(kAttnWarps * 32), st, pdl, a);
   return cudaErrorInvalidValue;
 }
 

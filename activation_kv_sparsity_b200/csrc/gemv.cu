@@ -1,35 +1,47 @@
 // Column-gathered bf16 GEMV with fp32 accumulation: the projection kernel of
 // every decode mode.
 //
-//   y[j] = sum over listed input channels c of x[c] * W[c][j]
+//   y[j] = s * sum over listed input channels c of v[c] * W[c][j]
 //
 // W is input-channel-major ([d_in][d_out]), so each selected channel is one
 // contiguous row and the activation-sparse projection (the ByteCross README's
 // projection branch, "Timing and quality on a GPU") reads exactly the rows of
 // the kept channels; dense mode is the same kernel over every row.
 //
-// Work split: CTA (tile, split) owns 256 output columns and a contiguous run
-// of `chunk` listed rows.  Each of its 8 warps streams every 8th row of the
-// run, one 16-byte vector per lane per row (512 contiguous bytes per warp and
-// row), with 8 rows in flight per warp.  Warps are reduced in shared memory;
-// splits are reduced by the last CTA of each column tile to arrive (an atomic
-// ticket, no spinning), which sums the partials in split order -- the result
-// is deterministic -- and applies the epilogue:
-//   STORE  y = r
-//   RESID  y += r (residual stream), optional copy for the layer trace
-//   QKV    raw output, rotary embedding of q and k heads, bf16 append of the
-//          new k and v at position pos, refresh of the page's key bounds
+// The GEMV input v is produced while staging, from the previous step's
+// output, so no separate kernel runs for it:
+//   NONE        v = x
+//   NORM        v = x * g, s = 1 / sqrt(mean(x^2) + eps)   (RMSNorm; the
+//               scale factors out of the sum and is applied to the partials)
+//   EMBED_NORM  the same with x = the token's bf16 embedding row; CTA 0 also
+//               initialises the residual stream with it
+//   SWIGLU      v = silu(gate) * up
+//
+// Work split: a column tile of 256 outputs is shared by the CTAs of one or
+// more thread-block clusters, and the tile's k listed rows are cut into one
+// contiguous run per CTA.  Each of a CTA's 8 warps streams every 8th row of
+// its run with 16 rows (8 KiB) in flight, 16 bytes per lane per row; warps are
+// reduced in shared memory.  The CTAs of a cluster then sum their partials
+// through distributed shared memory after a hardware cluster barrier (rank 0
+// reads them in rank order).  A tile split over several clusters adds one
+// stage through global scratch: each cluster's rank 0 writes its partial and
+// takes an atomic ticket; the last to arrive (no spinning) sums the clusters'
+// partials in order.  Both stages sum in a fixed order: deterministic.  The
+// CTA that holds the tile's complete sum applies the epilogue:
 #include "common.cuh"
 #include "kernels.h"
 
+#include <cooperative_groups.h>
 #include <math.h>
 #include <algorithm>
+
+namespace cg = cooperative_groups;
 
 namespace bc {
 
 constexpr int kGemvWarps = 8;
 constexpr int kGemvThreads = kGemvWarps * 32;
-constexpr int kGemvRowsInFlight = 8;
+constexpr int kRowsInFlight = 16;
 
 __device__ __forceinline__ void fma8(float* acc, float xv, const uint4& w) {
   acc[0] = fmaf(xv, bf16_lo(w.x), acc[0]);
@@ -42,13 +54,17 @@ __device__ __forceinline__ void fma8(float* acc, float xv, const uint4& w) {
   acc[7] = fmaf(xv, bf16_hi(w.w), acc[7]);
 }
 
-// Rotary embedding, bf16 append and key-bound refresh for one 256-column tile
-// of the q/k/v output.  Heads never straddle a tile (256 is a multiple of hd).
+// Rotary embedding, bf16 append and key-bound refresh for one TW-column tile
+// of the q/k/v output (v = this thread's column).  Heads never straddle a
+// tile (TW is a multiple of hd).  All threads pass the one barrier; threads
+// past the tile's width do nothing else.
+template <int TW>
 __device__ void qkv_epilogue(const QkvEpilogue& e, int col0, float v, float* s_v) {
   const int tid = threadIdx.x;
   const int col = col0 + tid;
-  s_v[tid] = v;
+  if (tid < TW) s_v[tid] = v;
   __syncthreads();
+  if (tid >= TW) return;
   const int hd = e.hd, half = hd >> 1;
   const int i = col % hd;
   const int qcols = e.Hq * hd, kcols = e.Hkv * hd;
@@ -68,62 +84,165 @@ __device__ void qkv_epilogue(const QkvEpilogue& e, int col0, float v, float* s_v
   }
   if (col < qcols) {
     e.q_out[col] = out;
-    return;
+  } else {
+    const int head = is_v ? (col - qcols - kcols) / hd : (col - qcols) / hd;
+    const int page = e.pos / kPage, slot = e.pos % kPage;
+    __nv_bfloat16* pg = e.kv_layer + ((size_t)head * e.Pmax + page) * (2 * kPage * hd);
+    const __nv_bfloat16 b = __float2bfloat16_rn(out);
+    if (is_v) {
+      pg[kPage * hd + slot * hd + i] = b;
+    } else {
+      pg[slot * hd + i] = b;
+      // bounds over the page's valid keys: earlier slots from the pool, this one
+      float mn = __bfloat162float(b), mx = mn;
+      #pragma unroll
+      for (int t = 0; t < kPage - 1; ++t) {
+        if (t < slot) {
+          const float kt = __bfloat162float(pg[t * hd + i]);
+          mn = fminf(mn, kt);
+          mx = fmaxf(mx, kt);
+        }
+      }
+      __nv_bfloat16* mt = e.meta_layer + ((size_t)head * e.Pmax + page) * (2 * hd);
+      mt[i] = __float2bfloat16_rn(mn);
+      mt[hd + i] = __float2bfloat16_rn(mx);
+    }
   }
-  const int head = is_v ? (col - qcols - kcols) / hd : (col - qcols) / hd;
-  const int page = e.pos / kPage, slot = e.pos % kPage;
-  __nv_bfloat16* pg = e.kv_layer + ((size_t)head * e.Pmax + page) * (2 * kPage * hd);
-  const __nv_bfloat16 b = __float2bfloat16_rn(out);
-  if (is_v) {
-    pg[kPage * hd + slot * hd + i] = b;
-    return;
-  }
-  pg[slot * hd + i] = b;
-  // bounds over the page's valid keys: earlier slots from the pool, this one
-  float mn = __bfloat162float(b), mx = mn;
-  for (int t = 0; t < slot; ++t) {
-    const float kt = __bfloat162float(pg[t * hd + i]);
-    mn = fminf(mn, kt);
-    mx = fmaxf(mx, kt);
-  }
-  __nv_bfloat16* mt = e.meta_layer + ((size_t)head * e.Pmax + page) * (2 * hd);
-  mt[i] = __float2bfloat16_rn(mn);
-  mt[hd + i] = __float2bfloat16_rn(mx);
 }
 
+__device__ __forceinline__ float prep_value(const GemvArgs& a, int c) {
+  switch (a.prep) {
+    case GP_NORM: return a.x[c] * bf16f(a.gain[c]);
+    case GP_EMBED_NORM: return bf16f(a.embed_row[c]) * bf16f(a.gain[c]);
+    case GP_SWIGLU: {
+      const float g = a.x[c], u = a.x[a.d_in + c];
+      return g / (1.0f + expf(-g)) * u;
+    }
+    default: return a.x[c];
+  }
+}
+
+// TW: columns per tile (256 or 128).  A row segment is TW*2 bytes read by
+// TW/8 lanes at 16 bytes each, so a warp instruction covers 32/(TW/8) rows.
+template <int TW>
 __global__ void __launch_bounds__(kGemvThreads, 2) k_gemv(GemvArgs a) {
+  constexpr int LPR = TW / 8;                      // lanes per row
+  constexpr int RPI = 32 / LPR;                    // rows per warp instruction
+  constexpr int ROWS_STEP = kGemvWarps * RPI;      // rows between a lane's consecutive rows
   extern __shared__ __align__(16) unsigned char smem[];
-  int* s_idx = reinterpret_cast<int*>(smem);
-  float* s_x = reinterpret_cast<float*>(smem + sizeof(int) * a.chunk);
-  __shared__ __align__(16) float s_red[kGemvWarps][kColTile];
+  __shared__ __align__(16) float s_red[kGemvWarps][TW];
+  __shared__ __align__(16) float s_part[TW];
+  __shared__ float s_v[kColTile];
+  __shared__ float s_sum[kGemvWarps];
   __shared__ int s_last;
+  cg::cluster_group cluster = cg::this_cluster();
 
-  const int tile = blockIdx.x, split = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int col0 = tile * kColTile;
-  const int r0 = split * a.chunk;
-  const int nr = min(a.k, r0 + a.chunk) - r0;
+  const int lrow = lane / LPR, lcol = lane % LPR;
+  const int t = blockIdx.y;                       // column tile
+  const int split = blockIdx.x;                   // run of rows: cluster * S + rank
+  const int nsplit = a.S * a.C;
+  const int r0 = (int)(((long long)a.k * split) / nsplit);
+  const int nr = (int)(((long long)a.k * (split + 1)) / nsplit) - r0;
+  const int col0 = t * TW;
+  int* s_idx = reinterpret_cast<int*>(smem);
+  float* s_x = reinterpret_cast<float*>(smem + sizeof(int) * a.max_rows);
+  const bool norm = a.prep == GP_NORM || a.prep == GP_EMBED_NORM;
+  const __nv_bfloat16* wcol = a.W + col0 + lcol * 8;
+  const size_t ld = (size_t)a.d_out;
+  const int my0 = warp * RPI + lrow;              // this lane's first row in the run
 
+  // Weights do not depend on the previous kernel: in dense mode issue this
+  // lane's first batch of rows before waiting for it.
+  uint4 w0[kRowsInFlight];
+  bool first_loaded = false;
+  if (!a.idx) {
+    #pragma unroll
+    for (int u = 0; u < kRowsInFlight; ++u) {
+      const int rr = my0 + u * ROWS_STEP;
+      w0[u] = rr < nr ? ld_stream(wcol + (size_t)(r0 + rr) * ld) : make_uint4(0, 0, 0, 0);
+    }
+    first_loaded = true;
+  }
   pdl_wait();
-  for (int r = tid; r < nr; r += kGemvThreads) {
-    const int c = a.idx ? a.idx[r0 + r] : r0 + r;
-    s_idx[r] = c;
-    s_x[r] = a.x[c];
+  pdl_trigger();
+  if (!first_loaded) {
+    // the warp's first 16*RPI listed rows: lane e fetches the index of batch
+    // element e = u*RPI + lrow, so the weight loads skip the staging barrier
+    int c = -1;
+    if (lane < kRowsInFlight * RPI) {
+      const int rr = warp * RPI + (lane % RPI) + (lane / RPI) * ROWS_STEP;
+      if (rr < nr) c = a.idx[r0 + rr];
+    }
+    #pragma unroll
+    for (int u = 0; u < kRowsInFlight; ++u) {
+      const int cu = __shfl_sync(0xffffffffu, c, u * RPI + lrow);
+      w0[u] = cu >= 0 ? ld_stream(wcol + (size_t)cu * ld) : make_uint4(0, 0, 0, 0);
+    }
+  }
+
+  // RMSNorm statistics over the whole input: independent loads, 4 in flight
+  float ss = 0.f;
+  if (norm) {
+    if (a.prep == GP_NORM) {
+      const float4* x4 = reinterpret_cast<const float4*>(a.x);
+      #pragma unroll 4
+      for (int c = tid; c < a.d_in / 4; c += kGemvThreads) {
+        const float4 v = x4[c];
+        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+      }
+    } else {
+      #pragma unroll 4
+      for (int c = tid; c < a.d_in; c += kGemvThreads) {
+        const float xv = bf16f(a.embed_row[c]);
+        ss = fmaf(xv, xv, ss);
+        if (blockIdx.x == 0 && blockIdx.y == 0) a.x_init[c] = xv;
+      }
+    }
+  }
+
+  // staging: 4 rows per thread per round, loads of a round in flight together
+  for (int rb = 0; rb < nr; rb += 4 * kGemvThreads) {
+    int cs[4];
+    #pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = rb + u * kGemvThreads + tid;
+      cs[u] = r < nr ? (a.idx ? a.idx[r0 + r] : r0 + r) : -1;
+    }
+    float vs[4];
+    #pragma unroll
+    for (int u = 0; u < 4; ++u) vs[u] = cs[u] >= 0 ? prep_value(a, cs[u]) : 0.f;
+    #pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = rb + u * kGemvThreads + tid;
+      if (r < nr) {
+        s_idx[r] = cs[u];
+        s_x[r] = vs[u];
+      }
+    }
+  }
+  if (norm) {
+    float v = ss;
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) s_sum[warp] = v;
   }
   __syncthreads();
-  pdl_trigger();
 
   float acc[8];
   #pragma unroll
   for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-  const __nv_bfloat16* wcol = a.W + col0 + lane * 8;
-  const size_t ld = (size_t)a.d_out;
-  for (int r = warp; r < nr; r += kGemvWarps * kGemvRowsInFlight) {
-    uint4 w[kGemvRowsInFlight];
-    float xv[kGemvRowsInFlight];
+  #pragma unroll
+  for (int u = 0; u < kRowsInFlight; ++u) {
+    const int rr = my0 + u * ROWS_STEP;
+    fma8(acc, rr < nr ? s_x[rr] : 0.f, w0[u]);
+  }
+  for (int r = my0 + ROWS_STEP * kRowsInFlight; r - lrow < nr; r += ROWS_STEP * kRowsInFlight) {
+    uint4 w[kRowsInFlight];
+    float xv[kRowsInFlight];
     #pragma unroll
-    for (int u = 0; u < kGemvRowsInFlight; ++u) {
-      const int rr = r + u * kGemvWarps;
+    for (int u = 0; u < kRowsInFlight; ++u) {
+      const int rr = r + u * ROWS_STEP;
       if (rr < nr) {
         w[u] = ld_stream(wcol + (size_t)s_idx[rr] * ld);
         xv[u] = s_x[rr];
@@ -133,75 +252,165 @@ __global__ void __launch_bounds__(kGemvThreads, 2) k_gemv(GemvArgs a) {
       }
     }
     #pragma unroll
-    for (int u = 0; u < kGemvRowsInFlight; ++u) fma8(acc, xv[u], w[u]);
+    for (int u = 0; u < kRowsInFlight; ++u) fma8(acc, xv[u], w[u]);
   }
-  float4* red4 = reinterpret_cast<float4*>(&s_red[warp][lane * 8]);
-  red4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  red4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-  __syncthreads();
-  float r = 0.f;
+  // lanes of the same columns (different rows) first, then the warps
   #pragma unroll
-  for (int w = 0; w < kGemvWarps; ++w) r += s_red[w][tid];
+  for (int o = LPR; o < 32; o <<= 1)
+    #pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+  if (lrow == 0) {
+    float4* red4 = reinterpret_cast<float4*>(&s_red[warp][lcol * 8]);
+    red4[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    red4[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+  __syncthreads();
+  float scale = 1.f;
+  if (norm) {
+    float tot = 0.f;
+    #pragma unroll
+    for (int w = 0; w < kGemvWarps; ++w) tot += s_sum[w];
+    scale = 1.0f / sqrtf(tot / (float)a.d_in + a.eps);
+  }
+  float r = 0.f;
+  if (tid < TW) {
+    #pragma unroll
+    for (int w = 0; w < kGemvWarps; ++w) r += s_red[w][tid];
+    s_part[tid] = r * scale;
+  }
 
-  const int col = col0 + tid;
-  if (a.n_chunks > 1) {
-    a.partial[(size_t)split * a.d_out + col] = r;
-    __threadfence();
+  // cluster stage: rank 0 sums the cluster's partials in rank order
+  cluster.sync();
+  const unsigned rank = cluster.block_rank();
+  bool have_total = false;
+  if (rank == 0) {
+    r = 0.f;
+    if (tid < TW)
+      for (int q = 0; q < a.S; ++q) r += cluster.map_shared_rank(s_part, q)[tid];
+    have_total = a.C == 1;
+  }
+  cluster.sync();                                  // peers' shared memory stays alive until read
+  if (rank != 0) return;
+
+  // global stage, when the tile is split over several clusters
+  if (a.C > 1) {
+    const int c = blockIdx.x / a.S;
+    if (tid < TW) a.partial[((size_t)t * kGemvMaxContrib + c) * TW + tid] = r;
     __syncthreads();
-    if (tid == 0) s_last = (atomicAdd(&a.counters[tile], 1u) == (unsigned)(a.n_chunks - 1));
+    if (tid == 0) {
+      __threadfence();   // the CTA's partials (ordered by the barrier) before the ticket
+      s_last = (atomicAdd(&a.counters[t], 1u) == (unsigned)(a.C - 1));
+    }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    r = 0.f;
-    for (int s = 0; s < a.n_chunks; ++s) r += ld_cg(&a.partial[(size_t)s * a.d_out + col]);
-    if (tid == 0) a.counters[tile] = 0u;
+    if (tid < TW) {
+      const float* pp = &a.partial[(size_t)t * kGemvMaxContrib * TW + tid];
+      float v[kGemvMaxContrib];
+      #pragma unroll
+      for (int q = 0; q < kGemvMaxContrib; ++q) v[q] = q < a.C ? ld_cg(pp + (size_t)q * TW) : 0.f;
+      r = 0.f;
+      #pragma unroll
+      for (int q = 0; q < kGemvMaxContrib; ++q) r += v[q];
+    }
+    if (tid == 0) a.counters[t] = 0u;
+    have_total = true;
   }
-  if (a.epi == EPI_STORE) {
-    a.y[col] = r;
-  } else if (a.epi == EPI_RESID) {
-    const float nx = a.y[col] + r;
-    a.y[col] = nx;
-    if (a.y_copy) a.y_copy[col] = nx;
-  } else {
-    a.y[col] = r;
-    __syncthreads();
-    qkv_epilogue(a.qkv, col0, r, &s_red[0][0]);
+  if (!have_total) return;
+  const int col = col0 + tid;
+  if (a.epi == EPI_QKV) {
+    if (tid < TW) a.y[col] = r;
+    qkv_epilogue<TW>(a.qkv, col0, r, s_v);
+  } else if (tid < TW) {
+    if (a.epi == EPI_STORE) {
+      a.y[col] = r;
+    } else {
+      const float nx = a.y[col] + r;
+      a.y[col] = nx;
+      if (a.y_copy) a.y_copy[col] = nx;
+    }
   }
 }
 
-void gemv_plan(int k, int d_out, int sms, int max_chunks, int* chunk, int* n_chunks) {
-  const int tiles = d_out / kColTile;
-  const int target = 2 * sms;                       // two resident CTAs per SM
-  int want = (target + tiles - 1) / tiles;
-  const int lo = (k + kGemvMaxChunkRows - 1) / kGemvMaxChunkRows;
-  const int hi = std::max(1, (k + 31) / 32);          // at least 32 rows per split
-  want = std::max(lo, std::min(want, hi));
-  want = std::max(1, std::min(want, max_chunks));
-  int c = (k + want - 1) / want;
-  *chunk = c;
-  *n_chunks = (k + c - 1) / c;
+static int g_max_cluster = 0;   // largest cluster size the GPU schedules for k_gemv
+
+template <int TW>
+static cudaError_t set_attrs() {
+  cudaError_t e = cudaFuncSetAttribute(k_gemv<TW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)(kGemvMaxPer * (sizeof(int) + sizeof(float))));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_gemv<TW>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+}
+
+static cudaError_t init_gemv_attrs() {
+  if (g_max_cluster) return cudaSuccess;
+  cudaError_t e = set_attrs<256>();
+  if (e == cudaSuccess) e = set_attrs<128>();
+  g_max_cluster = 8;
+  if (e == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16, 1);
+    cfg.blockDim = dim3(kGemvThreads);
+    cfg.dynamicSmemBytes = kGemvMaxPer * (sizeof(int) + sizeof(float));
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 16;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_gemv<256>, &cfg) == cudaSuccess && n > 0) g_max_cluster = 16;
+  }
+  cudaGetLastError();   // a refused query leaves no sticky state; clear the last-error slot
+  return cudaSuccess;
+}
+
+void gemv_plan(int k, int d_out, int sms, int* TW, int* S, int* C) {
+  init_gemv_attrs();
+  // 256-column tiles when there are enough of them, else 128-column tiles
+  int tw = 256;
+  if (d_out / 256 < 24 && d_out % 128 == 0) tw = 128;
+  const int tiles = d_out / tw;
+  // row runs per tile: about two CTAs per SM in all, at least 32 rows a run,
+  // at most kGemvMaxPer rows a run
+  int p = std::max(1, (2 * sms) / tiles);
+  p = std::min(p, std::max(1, k / 32));
+  p = std::max(p, (k + kGemvMaxPer - 1) / kGemvMaxPer);
+  // clusters of at most 8 (portable) unless a bigger one avoids the global stage
+  const int cap = std::max(1, g_max_cluster);
+  int s = 1;
+  while (s * 2 <= std::min(p, 8)) s *= 2;
+  if (p >= 16 && cap >= 16 && p < 32) s = 16;
+  // whole clusters only, never more row runs than planned (no extra wave);
+  // runs stay within the staging limit
+  int c = std::max(1, p / s);
+  while ((k + s * c - 1) / (s * c) > kGemvMaxPer) ++c;
+  c = std::min(c, kGemvMaxContrib);
+  *TW = tw;
+  *S = s;
+  *C = c;
 }
 
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st, bool pdl) {
-  const size_t smem = (size_t)a.chunk * (sizeof(int) + sizeof(float));
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemv, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(kGemvMaxChunkRows * (sizeof(int) + sizeof(float))));
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+  cudaError_t e = init_gemv_attrs();
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.d_out / kColTile, a.n_chunks);
+  cfg.gridDim = dim3(a.S * a.C, a.d_out / a.TW);
   cfg.blockDim = dim3(kGemvThreads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = (size_t)a.max_rows * (sizeof(int) + sizeof(float));
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_gemv, a);
+  cfg.numAttrs = pdl ? 2 : 1;
+  if (a.TW == 128) return cudaLaunchKernelEx(&cfg, k_gemv<128>, a);
+  return cudaLaunchKernelEx(&cfg, k_gemv<256>, a);
 }
 
 }  // namespace bc

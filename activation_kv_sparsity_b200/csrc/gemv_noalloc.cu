@@ -28,8 +28,8 @@
 namespace {
 
 constexpr int kNoAllocMaxDout = 32768;
-constexpr size_t kPartialBytes = 4ull * bc::kGemvMaxChunks * kNoAllocMaxDout;
-constexpr size_t kTicketBytes = 4ull * (kNoAllocMaxDout / bc::kColTile);
+constexpr size_t kPartialBytes = 4ull * bc::kGemvMaxContrib * kNoAllocMaxDout;
+constexpr size_t kTicketBytes = 4ull * (kNoAllocMaxDout / 128);   // one ticket per 128-column tile
 
 static __device__ __align__(256) unsigned char g_scratch[kPartialBytes + kTicketBytes];
 
@@ -76,8 +76,8 @@ extern "C" bc_status bc_gemv_noalloc(const void* W, int d_in, int d_out, const f
   }
   if (d_out > 0 && d_out % bc::kColTile == 0) {
     // the tickets must start at zero; a failed earlier call may have left some set
-    const size_t part = (4ull * bc::kGemvMaxChunks * d_out + 255) & ~size_t(255);
-    e = cudaMemsetAsync(static_cast<char*>(scratch) + part, 0, 4ull * (d_out / bc::kColTile),
+    const size_t part = (4ull * bc::kGemvMaxContrib * d_out + 255) & ~size_t(255);
+    e = cudaMemsetAsync(static_cast<char*>(scratch) + part, 0, 4ull * (d_out / 128),
                         static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
       bc::set_error("bc_gemv_noalloc: clearing the tickets failed");

@@ -12,6 +12,11 @@ void set_error(const char* msg);
 
 // ------------------------------------------------------------------ GEMV
 enum GemvEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_QKV = 2 };
+// How the GEMV input v is formed from x while staging (see gemv.cu).
+enum GemvPrep { GP_NONE = 0, GP_NORM = 1, GP_EMBED_NORM = 2, GP_SWIGLU = 3 };
+
+constexpr int kGemvMaxContrib = 64;   // clusters contributing to one column tile
+constexpr int kGemvMaxPer = 4096;     // listed rows per CTA (shared-memory staging)
 
 struct QkvEpilogue {
   int Hq, Hkv, hd, pos, Pmax;
@@ -24,57 +29,57 @@ struct QkvEpilogue {
 struct GemvArgs {
   const __nv_bfloat16* W;    // [d_in][d_out]
   int d_in, d_out;
-  const float* x;            // [d_in]
+  int prep;
+  const float* x;            // NONE: v; NORM: residual stream; SWIGLU: [gate | up] (2 d_in)
+  const __nv_bfloat16* gain; // NORM / EMBED_NORM
+  float eps;
+  const __nv_bfloat16* embed_row;  // EMBED_NORM
+  float* x_init;             // EMBED_NORM: residual stream written by CTA 0
   const int* idx;            // [k] ascending, or nullptr for all rows
   int k;
-  int chunk, n_chunks;       // rows per split, number of splits
-  float* partial;            // [n_chunks][d_out]
-  unsigned* counters;        // [d_out / 256], zero between launches
+  int TW;                    // columns per tile: 256 or 128
+  int S, C;                  // CTAs per cluster, clusters per column tile
+  int max_rows;              // rows of the longest run: ceil(k / (S*C))
+  float* partial;            // [d_out/TW][kGemvMaxContrib][TW] (C > 1 only)
+  unsigned* counters;        // [d_out / TW], zero between launches
   int epi;
   float* y;                  // STORE: y = r; RESID: y += r; QKV: y = r (raw)
   float* y_copy;             // RESID: optional copy of the updated y
   QkvEpilogue qkv;
 };
 
-// Grid shape for a GEMV of k rows and d_out columns on `sms` SMs.
-void gemv_plan(int k, int d_out, int sms, int max_chunks, int* chunk, int* n_chunks);
+// Shape of a GEMV of k listed rows and d_out columns on `sms` SMs: TW
+// columns per tile, S CTAs per cluster, C clusters per tile.
+void gemv_plan(int k, int d_out, int sms, int* TW, int* S, int* C);
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st, bool pdl);
-constexpr int kGemvMaxChunks = 64;
-constexpr int kGemvMaxChunkRows = 2048;
 
-// ------------------------------------------------------------------ selection / elementwise prep
-enum Prep { PREP_NONE = 0, PREP_NORM = 1, PREP_EMBED_NORM = 2, PREP_SWIGLU = 3 };
+// ------------------------------------------------------------------ activation select
+enum SelPrep { SP_NONE = 0, SP_NORM = 1, SP_EMBED_NORM = 2, SP_SWIGLU = 3 };
 
 struct SelectArgs {
   int prep;
-  int n;                          // vector length
-  int k;                          // kept count (used when do_select)
-  int do_select;
-  const float* v;                 // NONE: scored vector; NORM: x; SWIGLU: [gate | up] (2n)
+  int n;                          // vector length (<= kMaxSelect)
+  int k;                          // kept count
+  const float* x;                 // NONE: scored vector; NORM: x; SWIGLU: [gate | up] (2n)
   const __nv_bfloat16* gain;      // NORM / EMBED_NORM
-  float eps;
   const __nv_bfloat16* embed_row; // EMBED_NORM: the token's embedding row
-  float* x_out;                   // EMBED_NORM: residual stream initialised here
-  float* out;                     // NORM / SWIGLU output vector (the GEMV input)
+  float* x_init;                  // EMBED_NORM: residual stream initialised here
+  float* vout;                    // the ranked vector (trace), or nullptr
   int* idx;                       // [k] ascending
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl);
 
 // ------------------------------------------------------------------ KV pages
-struct PageScoreArgs {
+// Page scores, then (by the last CTA of each kv head) the page select.
+struct PageArgs {
   const float* q;                 // rotated queries [Hkv*G][hd]
   const __nv_bfloat16* meta;      // layer key bounds [Hkv][Pmax][2][hd]
-  int Hkv, G, hd, Pmax, P;
+  int Hkv, G, hd, Pmax, P, K, sinks, recent;
   float* scores;                  // [Hkv][Pmax]
-};
-cudaError_t launch_page_scores(const PageScoreArgs& a, cudaStream_t st, bool pdl);
-
-struct PageSelectArgs {
-  const float* scores;            // [Hkv][Pmax]
-  int Hkv, Pmax, P, K, sinks, recent;
   int* pages;                     // [Hkv][Pmax], first K ascending
+  unsigned* counters;             // [Hkv], zero between launches
 };
-cudaError_t launch_page_select(const PageSelectArgs& a, cudaStream_t st, bool pdl);
+cudaError_t launch_pages(const PageArgs& a, cudaStream_t st, bool pdl);
 
 // ------------------------------------------------------------------ attention
 struct AttnArgs {
@@ -85,6 +90,7 @@ struct AttnArgs {
   int splits, pages_per_split;
   float* part_o;                  // [Hkv*G][kMaxSplits][hd]
   float* part_ml;                 // [Hkv*G][kMaxSplits][2]
+  unsigned* counters;             // [Hkv], zero between launches
   float* out;                     // [Hkv*G][hd]
 };
 void attn_plan(int n_pages, int Hkv, int sms, int* splits, int* pps);
@@ -104,7 +110,9 @@ cudaError_t launch_kv_append(const KvAppendArgs& a, cudaStream_t st, bool pdl);
 struct LmHeadArgs {
   const __nv_bfloat16* W;         // [V][d]
   int V, d;
-  const float* xf;                // [d]
+  const float* x;                 // residual stream [d]
+  const __nv_bfloat16* gain;      // final RMSNorm gain [d]
+  float eps;
   float* logits;                  // [V]
 };
 cudaError_t launch_lmhead(const LmHeadArgs& a, int sms, cudaStream_t st, bool pdl);

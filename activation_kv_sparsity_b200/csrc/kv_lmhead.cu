@@ -72,17 +72,25 @@ cudaError_t launch_kv_append(const KvAppendArgs& a, cudaStream_t st, bool pdl) {
 }
 
 // ------------------------------------------------------------------ LM head
-// logits[r] = W[r] . xf, W output-major [V][d].  Each warp streams two rows
-// at a time, 16 bytes per lane per step; xf sits in shared memory.
+// logits[r] = s * W[r] . (x * g) with s = 1/sqrt(mean(x^2) + eps): the final
+// RMSNorm folded in (its scale factors out of every dot product).  W is
+// output-major [V][d].  Each warp streams two rows at a time, 16 bytes per
+// lane per step; x*g sits in shared memory.
 constexpr int kLmThreads = 256;
 
 __global__ void __launch_bounds__(kLmThreads) k_lmhead(LmHeadArgs a) {
   extern __shared__ __align__(16) float s_x[];
+  __shared__ float s_red[kLmThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31;
   pdl_wait();
   pdl_trigger();
-  for (int i = tid; i < a.d; i += kLmThreads) s_x[i] = a.xf[i];
-  __syncthreads();
+  float ss = 0.f;
+  for (int i = tid; i < a.d; i += kLmThreads) {
+    const float xv = a.x[i];
+    ss = fmaf(xv, xv, ss);
+    s_x[i] = xv * bf16f(a.gain[i]);
+  }
+  const float scale = 1.0f / sqrtf(block_sum<kLmThreads>(ss, s_red) / (float)a.d + a.eps);
   const int warps = gridDim.x * (kLmThreads / 32);
   const int gw = blockIdx.x * (kLmThreads / 32) + (tid >> 5);
   const int vecs = a.d / 8;            // 16-byte vectors per row
@@ -121,8 +129,8 @@ __global__ void __launch_bounds__(kLmThreads) k_lmhead(LmHeadArgs a) {
       s1 += __shfl_xor_sync(0xffffffffu, s1, o);
     }
     if (lane == 0) {
-      a.logits[r] = s0;
-      if (two) a.logits[r + 1] = s1;
+      a.logits[r] = s0 * scale;
+      if (two) a.logits[r + 1] = s1 * scale;
     }
   }
 }

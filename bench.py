@@ -194,8 +194,10 @@ def run_ours(args, rank, ws, local):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0 = time.time()
         e0.record(stream)
+        h0 = time.perf_counter()
         for i in range(steps):
             model.step(toks[warm + i], mode, logits, **kw)
+        host_enqueue[(mode, n)] = (time.perf_counter() - h0) * 1e3 / steps
         e1.record(stream)
         torch.cuda.synchronize()
         clocks.window(t0, time.time())
@@ -222,6 +224,7 @@ def run_ours(args, rank, ws, local):
 
     e2e = None
     cells = {}
+    host_enqueue = {}
     for n in contexts:
         if n == HEAD_CTX or (e2e is None and n == min(contexts)):
             e2e = time_e2e(n)
@@ -236,7 +239,8 @@ def run_ours(args, rank, ws, local):
             cells[(mode, n)] = dict(mode=mode, context=n, ms_per_step=round(ms, 4),
                                     tok_s=round(1000.0 / ms, 2), bytes_per_step=acc["impl_total_bytes"],
                                     gbs=round(gbs, 1), frac_of_measured_peak=round(gbs / peak, 4),
-                                    paper_bound=round(acc["bound"], 4), launches_per_step=launches // steps)
+                                    paper_bound=round(acc["bound"], 4), launches_per_step=launches // steps,
+                                    host_enqueue_ms=round(host_enqueue[(mode, n)], 4))
     for n in contexts:
         if ("dense", n) not in cells:
             continue
@@ -472,11 +476,14 @@ def run_kernel_only(args, local):
     g = torch.Generator(device=dev)
     g.manual_seed(0)
     stream = torch.cuda.current_stream(dev)
-    if args.only_kernel == "gemv_gateup":
+    if args.only_kernel in ("gemv_gateup", "gemv_gateup_dense"):
         d, d_out = cfg["hidden"], 2 * cfg["intermediate"]
         W = (torch.randn(d, d_out, generator=g, device=dev) * 0.02).to(torch.bfloat16)
-        k = math.ceil(0.5 * d - 1e-9)
-        idx = torch.sort(torch.randperm(d, device=dev, generator=g)[:k])[0].to(torch.int32)
+        if args.only_kernel == "gemv_gateup":
+            k = math.ceil(0.5 * d - 1e-9)
+            idx = torch.sort(torch.randperm(d, device=dev, generator=g)[:k])[0].to(torch.int32)
+        else:
+            k, idx = d, None
         x = torch.randn(d, generator=g, device=dev)
         y = torch.empty(d_out, device=dev)
         scratch = torch.zeros(bc.bc_gemv_scratch_bytes(d_out), dtype=torch.uint8, device=dev)
@@ -522,7 +529,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--modes", nargs="+", default=["dense", "act", "kv", "both"],
                     choices=["dense", "act", "kv", "both"])
-    ap.add_argument("--only-kernel", choices=("gemv_gateup", "attention"),
+    ap.add_argument("--only-kernel", choices=("gemv_gateup", "gemv_gateup_dense", "attention"),
                     help="time one kernel alone on a small case (profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -172,21 +172,23 @@ BC_API bc_status bc_decode_step_host(bc_model* m, int token, bc_mode mode, float
 
 /* Per-layer intermediates the last decode step left in the workspace, for
  * parity checks.  *ptr receives a device pointer into the workspace, *count
- * the number of valid elements (f32 unless noted).
- *   BC_TRACE_XN        RMSNorm output feeding q/k/v            [hidden]
+ * the number of valid elements (f32 unless noted; 0 when the step did not
+ * produce it).  The ranked vectors are exactly what the activation select
+ * ranked by magnitude; they exist only after an ACT or BOTH step.
+ *   BC_TRACE_XN        x * g, RMSNorm input times gain, ranked for q/k/v [hidden]
+ *                      (the norm's positive scale does not change the ranking)
  *   BC_TRACE_SEL_QKV   int32 selected channels, ascending       [k]
  *   BC_TRACE_Q         rotated queries                          [Hq hd]
- *   BC_TRACE_ATTN      attention output                         [Hq hd]
+ *   BC_TRACE_ATTN      attention output (ranked for o)          [Hq hd]
  *   BC_TRACE_SEL_O     int32                                    [k]
- *   BC_TRACE_XN2       RMSNorm output feeding gate/up           [hidden]
+ *   BC_TRACE_XN2       x * g ranked for gate/up                 [hidden]
  *   BC_TRACE_SEL_GU    int32                                    [k]
- *   BC_TRACE_H         silu(gate)*up                            [intermediate]
+ *   BC_TRACE_H         silu(gate)*up ranked for down            [intermediate]
  *   BC_TRACE_SEL_D     int32                                    [k]
  *   BC_TRACE_X         residual stream after the layer          [hidden]
  *   BC_TRACE_PAGE_SCORES f32 [Hkv][stride] (count = P, stride = Pmax)
  *   BC_TRACE_PAGES     int32 [Hkv][stride] kept pages ascending (count = K)
- *   BC_TRACE_QKV       raw q/k/v GEMV output before rotation    [(Hq+2Hkv) hd]
- * Selection traces have count 0 when the step did not select (dense). */
+ *   BC_TRACE_QKV       raw q/k/v GEMV output before rotation    [(Hq+2Hkv) hd] */
 typedef enum {
   BC_TRACE_XN = 0, BC_TRACE_SEL_QKV, BC_TRACE_Q, BC_TRACE_ATTN, BC_TRACE_SEL_O,
   BC_TRACE_XN2, BC_TRACE_SEL_GU, BC_TRACE_H, BC_TRACE_SEL_D, BC_TRACE_X,
@@ -204,8 +206,8 @@ BC_API bc_status bc_trace(const bc_model* m, int layer, bc_trace_kind kind,
  * idx: device int32 [k] ascending channel list, or NULL for all d_in
  * channels (then k must equal d_in); y: device f32 [d_out], overwritten.
  * scratch: device buffer of bc_gemv_scratch_bytes(d_out) bytes (split-K
- * partial sums and counters; counters must be zero before the first call,
- * and every call leaves them zero).  d_out must be a multiple of 256.
+ * partial sums and ticket counters; zero it before the first call: every
+ * call leaves the counters at zero).  d_out must be a multiple of 256.
  * stream: cudaStream_t.  Deterministic: the split-K partials are summed in a
  * fixed order. */
 BC_API size_t bc_gemv_scratch_bytes(int d_out);
@@ -243,7 +245,9 @@ BC_API bc_status bc_select_topk(const float* v, int n, int k, int* idx, void* st
  *          each row used, ascending), or NULL for pages 0..n_pages-1
  *   n_tok  valid tokens; the page n_tok/16 is partial
  *   out    device f32 [Hkv*G][hd]
- *   scratch  bc_attention_scratch_bytes(Hkv*G, hd) bytes */
+ *   scratch  bc_attention_scratch_bytes(Hkv*G, hd) bytes: split partials and
+ *            one ticket counter per kv head; zero it before the first call
+ *            (every call leaves the counters at zero) */
 BC_API size_t bc_attention_scratch_bytes(int n_q_heads, int head_dim);
 BC_API bc_status bc_attention(const float* q, const void* kv, int n_kv_heads, int group, int head_dim,
                               int Pmax, const int* pages, int n_pages, int n_tok,

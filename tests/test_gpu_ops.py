@@ -22,7 +22,7 @@ def _gen(seed):
 
 
 @pytest.mark.parametrize("d_in,d_out", [(512, 768), (512, 3584), (1792, 512), (4096, 6144), (4096, 4096),
-                                        (14336, 4096), (4096, 28672)])
+                                        (14336, 4096), (4096, 28672), (14336, 256), (4096, 512), (40, 256)])
 def test_gemv_dense_and_gathered(d_in, d_out):
     g = _gen(d_in * 7 + d_out)
     W = (torch.randn(d_in, d_out, generator=g) * 0.02).to(torch.bfloat16)
@@ -32,7 +32,9 @@ def test_gemv_dense_and_gathered(d_in, d_out):
     wb = bits(W)
     x64 = x.double().numpy()
     absmag = np.abs(x64) @ np.abs(od.bf16_to_f64(wb))     # summation error scale
-    for k in (None, 1, 37, d_in // 2 + 3, d_in):
+    for k in sorted({None, 1, 37, d_in // 2 + 3, d_in} - {None}) + [None]:
+        if k is not None and k > d_in:
+            continue
         if k is None:
             idx = None
             rows = None

@@ -27,7 +27,8 @@ def _inputs(d_in, d_out, k, seed):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("d_in,d_out,k", [(4096, 28672, 2048), (14336, 4096, 14336), (512, 768, 200)])
+@pytest.mark.parametrize("d_in,d_out,k", [(4096, 28672, 2048), (14336, 4096, 14336), (512, 768, 200),
+                                          (14336, 256, 14336), (14336, 512, 7000)])
 def test_noalloc_matches_gemv_twice(d_in, d_out, k):
     W, x, idx = _inputs(d_in, d_out, k, seed=d_out + k)
     scratch = torch.zeros(bc.bc_gemv_scratch_bytes(d_out), dtype=torch.uint8, device=DEV)
