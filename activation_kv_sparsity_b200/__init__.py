@@ -54,6 +54,7 @@ _SIGS = {
                                   C.POINTER(_P)]),
     "bc_model_destroy": (C.c_int, [_P]),
     "bc_set_stream": (C.c_int, [_P, _P]),
+    "bc_set_graphs": (C.c_int, [_P, C.c_int]),
     "bc_kv_length": (C.c_int, [_P]),
     "bc_launch_count": (C.c_longlong, [_P]),
     "bc_kv_reset": (C.c_int, [_P, C.c_int]),
@@ -152,6 +153,9 @@ class Model:
 
     def __len__(self):
         return bc_kv_length(self.h)
+
+    def set_graphs(self, enable: bool):
+        check(bc_set_graphs(self.h, 1 if enable else 0), "bc_set_graphs")
 
     def launches(self) -> int:
         return bc_launch_count(self.h)

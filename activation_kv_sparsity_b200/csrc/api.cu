@@ -10,6 +10,7 @@
 #include <string.h>
 #include <algorithm>
 #include <string>
+#include <vector>
 
 using namespace bc;
 
@@ -162,7 +163,44 @@ struct bc_model {
   int last_k[4];       // kept channels per site (0 = no selection)
   int last_P, last_K;  // pages after the append, kept pages (0 = no selection)
   bool last_act;       // the last step ranked activations (XN, XN2, H traces valid)
+  // CUDA graphs of the step, one per step configuration
+  bool use_graphs;
+  cudaStream_t cap_stream;                 // private stream the steps are captured on
+  std::vector<struct StepGraph*> graphs;
 };
+
+// A kernel node of a captured step whose arguments change from step to step.
+enum NodeKind { NK_QKV = 0, NK_SEL_EMBED, NK_PAGES, NK_ATTN, NK_LMHEAD };
+struct NodeRec {
+  cudaGraphNode_t node;
+  int kind, layer;
+  cudaKernelNodeParams kp;   // function and launch shape read back from the graph
+  union {
+    GemvArgs g;
+    SelectArgs s;
+    PageArgs p;
+    AttnArgs a;
+    LmHeadArgs lm;
+  } args;
+};
+
+// A captured decode step for one (mode, rp, rkv, sinks, recent).
+struct StepGraph {
+  bc_mode mode;
+  float rp, rkv;
+  int sinks, recent;
+  cudaGraph_t graph;
+  cudaGraphExec_t exec;
+  std::vector<NodeRec> nodes;
+  long long launches;
+};
+
+static void destroy_graph(StepGraph* g) {
+  if (!g) return;
+  if (g->exec) cudaGraphExecDestroy(g->exec);
+  if (g->graph) cudaGraphDestroy(g->graph);
+  delete g;
+}
 
 template <typename T>
 static T* at(const bc_model* m, size_t off) { return reinterpret_cast<T*>(m->ws + off); }
@@ -205,6 +243,8 @@ extern "C" bc_status bc_model_create(const bc_config* cfg, const bc_weights* w, 
   memset(m->last_k, 0, sizeof m->last_k);
   m->last_P = m->last_K = 0;
   m->last_act = false;
+  m->use_graphs = true;
+  m->cap_stream = nullptr;
   cudaError_t e = cudaMemsetAsync(m->ws + lay.counters, 0, counter_bytes(cfg, lay), m->stream);
   if (e != cudaSuccess) {
     delete m;
@@ -215,7 +255,16 @@ extern "C" bc_status bc_model_create(const bc_config* cfg, const bc_weights* w, 
 }
 
 extern "C" bc_status bc_model_destroy(bc_model* m) {
+  if (!m) return BC_OK;
+  for (StepGraph* g : m->graphs) destroy_graph(g);
+  if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
   delete m;
+  return BC_OK;
+}
+
+extern "C" bc_status bc_set_graphs(bc_model* m, int enable) {
+  if (!m) return fail(BC_EINVAL, "null model");
+  m->use_graphs = enable != 0;
   return BC_OK;
 }
 
@@ -279,7 +328,7 @@ static bc_status check_step(const bc_model* m, bc_mode mode, float rp, float rkv
 
 static cudaError_t step_select(bc_model* m, int prep, int n, int k, const float* x,
                                const __nv_bfloat16* gain, const __nv_bfloat16* emb, float* x_init,
-                               float* vout, int* idx) {
+                               float* vout, int* idx, SelectArgs* out_args) {
   SelectArgs s;
   s.prep = prep;
   s.n = n;
@@ -290,6 +339,7 @@ static cudaError_t step_select(bc_model* m, int prep, int n, int k, const float*
   s.x_init = x_init;
   s.vout = vout;
   s.idx = idx;
+  if (out_args) *out_args = s;
   return launch_select(s, m->stream, true);
 }
 
@@ -300,7 +350,7 @@ static unsigned* gemv_counters(bc_model* m, int site) {
 static cudaError_t step_gemv(bc_model* m, int site, const __nv_bfloat16* W, int d_in, int d_out, int prep,
                              const float* x, const __nv_bfloat16* gain, const __nv_bfloat16* emb,
                              float* x_init, const int* idx, int k, int epi, float* y, float* y_copy,
-                             const QkvEpilogue* qe) {
+                             const QkvEpilogue* qe, GemvArgs* out_args) {
   GemvArgs g;
   memset(&g, 0, sizeof g);
   g.W = W;
@@ -322,11 +372,80 @@ static cudaError_t step_gemv(bc_model* m, int site, const __nv_bfloat16* W, int 
   g.y = y;
   g.y_copy = y_copy;
   if (qe) g.qkv = *qe;
+  if (out_args) *out_args = g;
   return launch_gemv(g, m->stream, true);
 }
 
+// The kernel node the last launch added to a stream being captured.
+static cudaGraphNode_t captured_node(cudaStream_t st) {
+  cudaStreamCaptureStatus status;
+  const cudaGraphNode_t* deps = nullptr;
+  size_t n = 0;
+  if (cudaStreamGetCaptureInfo(st, &status, nullptr, nullptr, &deps, &n) != cudaSuccess) return nullptr;
+  return (status == cudaStreamCaptureStatusActive && n == 1) ? deps[0] : nullptr;
+}
+
+template <typename A>
+static bool record(std::vector<NodeRec>* rec, cudaStream_t st, int kind, int layer, const A& args) {
+  if (!rec) return true;
+  NodeRec r;
+  memset(&r, 0, sizeof r);
+  r.node = captured_node(st);
+  if (!r.node) return false;
+  r.kind = kind;
+  r.layer = layer;
+  memcpy(&r.args, &args, sizeof(A));
+  rec->push_back(r);
+  return true;
+}
+
+// Per-step values every mode derives from the position.
+struct StepShape {
+  int pos, n_tok, P, K, splits, pps;
+  int k_qkv, k_o, k_gu, k_d;
+};
+
+static StepShape step_shape(const bc_model* m, bc_mode mode, float rp, float rkv, int sinks, int recent) {
+  const bc_config& c = m->cfg;
+  const bool act = mode == BC_ACT || mode == BC_BOTH;
+  const bool kvs = mode == BC_KV || mode == BC_BOTH;
+  StepShape sh;
+  sh.pos = m->n;
+  sh.n_tok = sh.pos + 1;
+  sh.P = (sh.n_tok + kPage - 1) / kPage;
+  sh.K = sh.P;
+  if (kvs) {
+    const int sink_end = std::min(sinks, sh.P), rec_begin = std::max(sh.P - recent, 0);
+    const int n_forced = sink_end + (sh.P - std::max(rec_begin, sink_end));
+    const int want = (int)std::min<double>(sh.P, ceil((double)rkv * sh.P - 1e-9));
+    sh.K = std::max(n_forced, want);
+  }
+  attn_plan(sh.K, c.n_kv_heads, m->sms, &sh.splits, &sh.pps);
+  sh.k_qkv = act ? keep_count(rp, c.hidden) : c.hidden;
+  sh.k_o = act ? keep_count(rp, m->lay.hq) : m->lay.hq;
+  sh.k_gu = act ? keep_count(rp, c.hidden) : c.hidden;
+  sh.k_d = act ? keep_count(rp, c.intermediate) : c.intermediate;
+  return sh;
+}
+
+static void commit_step(bc_model* m, bc_mode mode, const StepShape& sh, long long launches) {
+  const bool act = mode == BC_ACT || mode == BC_BOTH;
+  const bool kvs = mode == BC_KV || mode == BC_BOTH;
+  m->launches += launches;
+  m->n = sh.n_tok;
+  m->last_k[0] = act ? sh.k_qkv : 0;
+  m->last_k[1] = act ? sh.k_o : 0;
+  m->last_k[2] = act ? sh.k_gu : 0;
+  m->last_k[3] = act ? sh.k_d : 0;
+  m->last_act = act;
+  m->last_P = sh.P;
+  m->last_K = kvs ? sh.K : 0;
+}
+
+// Enqueues one decode step on m->stream (launching, or recording into a
+// capture when rec is given).  Returns the number of kernels in *launches.
 static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, float rkv, int sinks,
-                              int recent, float* logits) {
+                              int recent, float* logits, std::vector<NodeRec>* rec, long long* n_launch) {
   const bc_config& c = m->cfg;
   const Layout& y = m->lay;
   const bool act = mode == BC_ACT || mode == BC_BOTH;
@@ -334,19 +453,10 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
   const int L = c.n_layers, d = c.hidden, f = c.intermediate, hd = c.head_dim;
   const int Hq = c.n_heads, Hkv = c.n_kv_heads, G = Hq / Hkv;
   const int hq = y.hq, nqkv = y.nqkv, Pmax = y.Pmax;
-  const int pos = m->n, n_tok = pos + 1;
-  const int P = (n_tok + kPage - 1) / kPage;
-  int K = P;
-  if (kvs) {
-    const int sink_end = std::min(sinks, P), rec_begin = std::max(P - recent, 0);
-    const int n_forced = sink_end + (P - std::max(rec_begin, sink_end));
-    const int want = (int)std::min<double>(P, ceil((double)rkv * P - 1e-9));
-    K = std::max(n_forced, want);
-  }
-  const int k_qkv = act ? keep_count(rp, d) : d;
-  const int k_o = act ? keep_count(rp, hq) : hq;
-  const int k_gu = act ? keep_count(rp, d) : d;
-  const int k_d = act ? keep_count(rp, f) : f;
+  const StepShape sh = step_shape(m, mode, rp, rkv, sinks, recent);
+  const int pos = sh.pos, n_tok = sh.n_tok, P = sh.P, K = sh.K;
+  const int k_qkv = sh.k_qkv, k_o = sh.k_o, k_gu = sh.k_gu, k_d = sh.k_d;
+  cudaStream_t st = m->stream;
 
   const __nv_bfloat16* emb = static_cast<const __nv_bfloat16*>(m->w.embed) + (size_t)token * d;
   const __nv_bfloat16* attn_norm = static_cast<const __nv_bfloat16*>(m->w.attn_norm);
@@ -361,8 +471,7 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
   unsigned* att_counters = gemv_counters(m, 4);
   unsigned* page_counters = att_counters + Hkv;
 
-  int splits, pps;
-  attn_plan(K, Hkv, m->sms, &splits, &pps);
+  const int splits = sh.splits, pps = sh.pps;
   long long launches = 0;
 
   for (int l = 0; l < L; ++l) {
@@ -390,8 +499,10 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
     // append and page bounds in the epilogue) -> [page scores + select] ->
     // split-K attention with fused combine
     if (act) {
-      BC_CUDA(step_select(m, first ? SP_EMBED_NORM : SP_NORM, d, k_qkv, x, g_attn, emb, x, xn, s_qkv),
+      SelectArgs sa;
+      BC_CUDA(step_select(m, first ? SP_EMBED_NORM : SP_NORM, d, k_qkv, x, g_attn, emb, x, xn, s_qkv, &sa),
               "select qkv");
+      if (first && !record(rec, st, NK_SEL_EMBED, l, sa)) return fail(BC_ECUDA, "capture: no node");
       ++launches;
     }
     QkvEpilogue qe;
@@ -404,12 +515,15 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
     qe.q_out = q;
     qe.kv_layer = kvl;
     qe.meta_layer = metal;
+    GemvArgs ga;
     BC_CUDA(step_gemv(m, 0, wqkv + (size_t)l * d * nqkv, d, nqkv, first ? GP_EMBED_NORM : GP_NORM, x, g_attn,
-                      emb, x, act ? s_qkv : nullptr, k_qkv, EPI_QKV, qkv, nullptr, &qe), "gemv qkv");
+                      emb, x, act ? s_qkv : nullptr, k_qkv, EPI_QKV, qkv, nullptr, &qe, &ga), "gemv qkv");
+    if (!record(rec, st, NK_QKV, l, ga)) return fail(BC_ECUDA, "capture: no node");
     ++launches;
     if (kvs) {
       PageArgs pa{q, metal, Hkv, G, hd, Pmax, P, K, sinks, recent, pscore, pages, page_counters};
-      BC_CUDA(launch_pages(pa, m->stream, true), "page scores and select");
+      BC_CUDA(launch_pages(pa, st, true), "page scores and select");
+      if (!record(rec, st, NK_PAGES, l, pa)) return fail(BC_ECUDA, "capture: no node");
       ++launches;
     }
     AttnArgs aa;
@@ -428,47 +542,156 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
     aa.part_ml = at<float>(m, y.part_ml);
     aa.counters = att_counters;
     aa.out = attn;
-    BC_CUDA(launch_attention(aa, m->stream, true), "attention");
+    BC_CUDA(launch_attention(aa, st, true), "attention");
+    if (!record(rec, st, NK_ATTN, l, aa)) return fail(BC_ECUDA, "capture: no node");
     ++launches;
     if (act) {
-      BC_CUDA(step_select(m, SP_NONE, hq, k_o, attn, nullptr, nullptr, nullptr, nullptr, s_o), "select o");
+      BC_CUDA(step_select(m, SP_NONE, hq, k_o, attn, nullptr, nullptr, nullptr, nullptr, s_o, nullptr),
+              "select o");
       ++launches;
     }
     BC_CUDA(step_gemv(m, 1, wo + (size_t)l * hq * d, hq, d, GP_NONE, attn, nullptr, nullptr, nullptr,
-                      act ? s_o : nullptr, k_o, EPI_RESID, x, nullptr, nullptr), "gemv o");
+                      act ? s_o : nullptr, k_o, EPI_RESID, x, nullptr, nullptr, nullptr), "gemv o");
     ++launches;
     // feed-forward block: [select] -> gate/up GEMV (RMSNorm folded in) ->
     // [select] -> down GEMV (SwiGLU folded in) + residual
     if (act) {
-      BC_CUDA(step_select(m, SP_NORM, d, k_gu, x, g_mlp, nullptr, nullptr, xn2, s_gu), "select gate/up");
+      BC_CUDA(step_select(m, SP_NORM, d, k_gu, x, g_mlp, nullptr, nullptr, xn2, s_gu, nullptr),
+              "select gate/up");
       ++launches;
     }
     BC_CUDA(step_gemv(m, 2, wgu + (size_t)l * d * 2 * f, d, 2 * f, GP_NORM, x, g_mlp, nullptr, nullptr,
-                      act ? s_gu : nullptr, k_gu, EPI_STORE, gu, nullptr, nullptr), "gemv gate/up");
+                      act ? s_gu : nullptr, k_gu, EPI_STORE, gu, nullptr, nullptr, nullptr), "gemv gate/up");
     ++launches;
     if (act) {
-      BC_CUDA(step_select(m, SP_SWIGLU, f, k_d, gu, nullptr, nullptr, nullptr, hmid, s_d), "select down");
+      BC_CUDA(step_select(m, SP_SWIGLU, f, k_d, gu, nullptr, nullptr, nullptr, hmid, s_d, nullptr),
+              "select down");
       ++launches;
     }
     BC_CUDA(step_gemv(m, 3, wd + (size_t)l * f * d, f, d, GP_SWIGLU, gu, nullptr, nullptr, nullptr,
-                      act ? s_d : nullptr, k_d, EPI_RESID, x, xo, nullptr), "gemv down");
+                      act ? s_d : nullptr, k_d, EPI_RESID, x, xo, nullptr, nullptr), "gemv down");
     ++launches;
   }
   LmHeadArgs lm{static_cast<const __nv_bfloat16*>(m->w.lm_head), c.vocab, d, x,
                 static_cast<const __nv_bfloat16*>(m->w.final_norm), c.rms_eps, logits};
-  BC_CUDA(launch_lmhead(lm, m->sms, m->stream, true), "lm head");
+  BC_CUDA(launch_lmhead(lm, m->sms, st, true), "lm head");
+  if (!record(rec, st, NK_LMHEAD, 0, lm)) return fail(BC_ECUDA, "capture: no node");
   ++launches;
-
-  m->launches += launches;
-  m->n = n_tok;
-  m->last_k[0] = act ? k_qkv : 0;
-  m->last_k[1] = act ? k_o : 0;
-  m->last_k[2] = act ? k_gu : 0;
-  m->last_k[3] = act ? k_d : 0;
-  m->last_act = act;
-  m->last_P = P;
-  m->last_K = kvs ? K : 0;
+  *n_launch = launches;
   return BC_OK;
+}
+
+// Captures the step for this configuration on the private stream.
+static bc_status capture_step(bc_model* m, int token, bc_mode mode, float rp, float rkv, int sinks,
+                              int recent, float* logits, StepGraph** out) {
+  if (!m->cap_stream) BC_CUDA(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking), "capture stream");
+  StepGraph* g = new StepGraph();
+  g->mode = mode;
+  g->rp = rp;
+  g->rkv = rkv;
+  g->sinks = sinks;
+  g->recent = recent;
+  g->graph = nullptr;
+  g->exec = nullptr;
+  cudaStream_t user = m->stream;
+  m->stream = m->cap_stream;
+  cudaError_t e = cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal);
+  bc_status s = BC_OK;
+  if (e == cudaSuccess) s = enqueue_step(m, token, mode, rp, rkv, sinks, recent, logits, &g->nodes, &g->launches);
+  cudaError_t e2 = cudaStreamEndCapture(m->cap_stream, &g->graph);
+  m->stream = user;
+  if (e != cudaSuccess || s != BC_OK || e2 != cudaSuccess) {
+    destroy_graph(g);
+    cudaGetLastError();
+    return fail(BC_ECUDA, "capturing the step failed (%s)", cudaGetErrorString(e != cudaSuccess ? e : e2));
+  }
+  e = cudaGraphInstantiate(&g->exec, g->graph, 0);
+  for (size_t i = 0; e == cudaSuccess && i < g->nodes.size(); ++i)
+    e = cudaGraphKernelNodeGetParams(g->nodes[i].node, &g->nodes[i].kp);
+  if (e != cudaSuccess) {
+    destroy_graph(g);
+    return cuda_fail(e, "instantiating the step graph");
+  }
+  *out = g;
+  return BC_OK;
+}
+
+// Points the recorded nodes at this step's position, token, page counts and
+// logits buffer, then launches the graph on the model's stream.
+static cudaError_t launch_step_graph(bc_model* m, StepGraph* g, int token, const StepShape& sh, float* logits) {
+  const bc_config& c = m->cfg;
+  const __nv_bfloat16* emb = static_cast<const __nv_bfloat16*>(m->w.embed) + (size_t)token * c.hidden;
+  for (NodeRec& r : g->nodes) {
+    cudaKernelNodeParams kp = r.kp;
+    void* argp = &r.args;
+    switch (r.kind) {
+      case NK_QKV:
+        r.args.g.qkv.pos = sh.pos;
+        if (r.args.g.prep == GP_EMBED_NORM) r.args.g.embed_row = emb;
+        break;
+      case NK_SEL_EMBED:
+        r.args.s.embed_row = emb;
+        break;
+      case NK_PAGES:
+        r.args.p.P = sh.P;
+        r.args.p.K = sh.K;
+        kp.gridDim = pages_grid(r.args.p);
+        kp.sharedMemBytes = (unsigned)pages_smem(r.args.p);
+        break;
+      case NK_ATTN:
+        r.args.a.n_pages = sh.K;
+        r.args.a.n_tok = sh.n_tok;
+        r.args.a.splits = sh.splits;
+        r.args.a.pages_per_split = sh.pps;
+        kp.gridDim = dim3(sh.splits, c.n_kv_heads);
+        break;
+      case NK_LMHEAD:
+        r.args.lm.logits = logits;
+        break;
+    }
+    kp.kernelParams = &argp;
+    kp.extra = nullptr;
+    cudaError_t e = cudaGraphExecKernelNodeSetParams(g->exec, r.node, &kp);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaGraphLaunch(g->exec, m->stream);
+}
+
+static bc_status run_step(bc_model* m, int token, bc_mode mode, float rp, float rkv, int sinks, int recent,
+                          float* logits) {
+  const StepShape sh = step_shape(m, mode, rp, rkv, sinks, recent);
+  if (m->use_graphs) {
+    StepGraph* g = nullptr;
+    for (StepGraph* c : m->graphs)
+      if (c->mode == mode && c->rp == rp && c->rkv == rkv && c->sinks == sinks && c->recent == recent) g = c;
+    if (g) {
+      cudaError_t e = launch_step_graph(m, g, token, sh, logits);
+      if (e == cudaSuccess) {
+        commit_step(m, mode, sh, g->launches);
+        return BC_OK;
+      }
+      // an update the graph refused: drop it, run directly, capture again next time
+      cudaGetLastError();
+      m->graphs.erase(std::find(m->graphs.begin(), m->graphs.end(), g));
+      destroy_graph(g);
+    } else if (m->launches > 0) {
+      // the kernels' attributes are set up by an earlier direct step: capture now
+      if (capture_step(m, token, mode, rp, rkv, sinks, recent, logits, &g) == BC_OK) {
+        m->graphs.push_back(g);
+        if (launch_step_graph(m, g, token, sh, logits) == cudaSuccess) {
+          commit_step(m, mode, sh, g->launches);
+          return BC_OK;
+        }
+        cudaGetLastError();
+        m->graphs.pop_back();
+        destroy_graph(g);
+      }
+    }
+  }
+  long long launches = 0;
+  bc_status s = enqueue_step(m, token, mode, rp, rkv, sinks, recent, logits, nullptr, &launches);
+  if (s == BC_OK) commit_step(m, mode, sh, launches);
+  return s;
 }
 
 extern "C" bc_status bc_decode_step(bc_model* m, int token, bc_mode mode, float rp, float rkv,
@@ -477,7 +700,7 @@ extern "C" bc_status bc_decode_step(bc_model* m, int token, bc_mode mode, float 
   if (s != BC_OK) return s;
   if (!logits) return fail(BC_EINVAL, "null logits");
   if (token < 0 || token >= m->cfg.vocab) return fail(BC_EINVAL, "token %d outside the vocabulary", token);
-  return enqueue_step(m, token, mode, rp, rkv, sinks, recent, logits);
+  return run_step(m, token, mode, rp, rkv, sinks, recent, logits);
 }
 
 extern "C" bc_status bc_decode_step_host(bc_model* m, int token, bc_mode mode, float rp, float rkv,
@@ -487,7 +710,7 @@ extern "C" bc_status bc_decode_step_host(bc_model* m, int token, bc_mode mode, f
   if (!logits_host) return fail(BC_EINVAL, "null logits");
   if (token < 0 || token >= m->cfg.vocab) return fail(BC_EINVAL, "token %d outside the vocabulary", token);
   float* dev = at<float>(m, m->lay.logits);
-  s = enqueue_step(m, token, mode, rp, rkv, sinks, recent, dev);
+  s = run_step(m, token, mode, rp, rkv, sinks, recent, dev);
   if (s != BC_OK) return s;
   BC_CUDA(cudaMemcpyAsync(logits_host, dev, sizeof(float) * m->cfg.vocab, cudaMemcpyDeviceToHost, m->stream),
           "bc_decode_step_host: copy logits");

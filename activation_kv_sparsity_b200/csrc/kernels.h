@@ -80,6 +80,9 @@ struct PageArgs {
   unsigned* counters;             // [Hkv], zero between launches
 };
 cudaError_t launch_pages(const PageArgs& a, cudaStream_t st, bool pdl);
+// Launch shape of the page kernel for P pages (graph node updates).
+dim3 pages_grid(const PageArgs& a);
+size_t pages_smem(const PageArgs& a);
 
 // ------------------------------------------------------------------ attention
 struct AttnArgs {

@@ -359,8 +359,14 @@ __global__ void __launch_bounds__(kPageThreads) k_pages(PageArgs a) {
       a.pages + (size_t)h * a.Pmax, sm, lo, hi);
 }
 
-cudaError_t launch_pages(const PageArgs& a, cudaStream_t st, bool pdl) {
+dim3 pages_grid(const PageArgs& a) {
   const int ppc = (kPageThreads / 32) * (32 / (a.hd / 8)) * 4;
+  return dim3((a.P + ppc - 1) / ppc, a.Hkv);
+}
+
+size_t pages_smem(const PageArgs& a) { return (size_t)a.P * sizeof(uint32_t); }
+
+cudaError_t launch_pages(const PageArgs& a, cudaStream_t st, bool pdl) {
   static bool attr_done = false;
   if (!attr_done) {
     const int smem = kMaxSelect * (int)sizeof(uint32_t);
@@ -370,9 +376,9 @@ cudaError_t launch_pages(const PageArgs& a, cudaStream_t st, bool pdl) {
     attr_done = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((a.P + ppc - 1) / ppc, a.Hkv);
+  cfg.gridDim = pages_grid(a);
   cfg.blockDim = dim3(kPageThreads);
-  cfg.dynamicSmemBytes = (size_t)a.P * sizeof(uint32_t);
+  cfg.dynamicSmemBytes = pages_smem(a);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -115,6 +115,16 @@ BC_API bc_status bc_model_destroy(bc_model* m);
 /* Stream used by later calls on this model. */
 BC_API bc_status bc_set_stream(bc_model* m, void* stream);
 
+/* Decode steps through CUDA graphs (enable != 0, the default) or through
+ * direct launches.  With graphs on, the first step of a configuration
+ * (mode, rp, rkv, sinks, recent) launches directly; the next one captures the
+ * step on a private stream of the library (created on first use) into a
+ * graph, and every later step of that configuration updates the few kernel
+ * nodes that depend on the position, token, page counts and logits buffer
+ * and launches the graph on the model's stream.  Results are identical
+ * either way (the same kernels with the same arguments).  Host-only. */
+BC_API bc_status bc_set_graphs(bc_model* m, int enable);
+
 /* Number of cached tokens. */
 BC_API int bc_kv_length(const bc_model* m);
 

@@ -94,6 +94,30 @@ def test_steps_are_deterministic(tiny):
     assert torch.equal(res[0], res[1])
 
 
+@pytest.mark.parametrize("mode", ["dense", "act", "kv", "both"])
+def test_graph_steps_equal_direct_steps(tiny, mode):
+    """Steps replayed from a captured CUDA graph (nodes updated per step) give
+    the same logits, bit for bit, as direct launches, across page boundaries
+    (the page count and the attention grid change between steps)."""
+    cfg = tiny["cfg"]
+    start = N_CTX - 20                       # crosses positions 2032 and 2048 (page boundaries)
+    outs = {}
+    for graphs in (False, True):
+        m = _model(tiny)
+        m.set_graphs(graphs)
+        m.reset(start)
+        logits = torch.empty(cfg["vocab"], device=DEV)
+        seq = []
+        for tok in tokens(24, cfg["vocab"], seed=9):
+            m.step(tok, mode, logits, **KW)
+            seq.append(logits.clone())
+        torch.cuda.synchronize()
+        outs[graphs] = seq
+        m.close()
+    for i, (a, b) in enumerate(zip(outs[False], outs[True])):
+        assert torch.equal(a, b), (mode, i)
+
+
 def _meta(m, cfg, max_ctx):
     Pmax = -(-max_ctx // 16)
     return m.meta_pool.view(torch.bfloat16).view(cfg["n_layers"], cfg["n_kv_heads"], Pmax, 2, cfg["head_dim"])
