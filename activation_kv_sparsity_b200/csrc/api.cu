@@ -170,7 +170,7 @@ struct bc_model {
 };
 
 // A kernel node of a captured step whose arguments change from step to step.
-enum NodeKind { NK_QKV = 0, NK_SEL_EMBED, NK_PAGES, NK_ATTN, NK_LMHEAD };
+enum NodeKind { NK_QKV = 0, NK_SEL_EMBED, NK_PAGES, NK_PAGE_SEL, NK_ATTN, NK_LMHEAD };
 struct NodeRec {
   cudaGraphNode_t node;
   int kind, layer;
@@ -522,9 +522,11 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
     ++launches;
     if (kvs) {
       PageArgs pa{q, metal, Hkv, G, hd, Pmax, P, K, sinks, recent, pscore, pages, page_counters};
-      BC_CUDA(launch_pages(pa, st, true), "page scores and select");
+      BC_CUDA(launch_page_scores(pa, st, true), "page scores");
       if (!record(rec, st, NK_PAGES, l, pa)) return fail(BC_ECUDA, "capture: no node");
-      ++launches;
+      BC_CUDA(launch_page_select(pa, st, true), "page select");
+      if (!record(rec, st, NK_PAGE_SEL, l, pa)) return fail(BC_ECUDA, "capture: no node");
+      launches += 2;
     }
     AttnArgs aa;
     aa.q = q;
@@ -636,7 +638,10 @@ static cudaError_t launch_step_graph(bc_model* m, StepGraph* g, int token, const
         r.args.p.P = sh.P;
         r.args.p.K = sh.K;
         kp.gridDim = pages_grid(r.args.p);
-        kp.sharedMemBytes = (unsigned)pages_smem(r.args.p);
+        break;
+      case NK_PAGE_SEL:
+        r.args.p.P = sh.P;
+        r.args.p.K = sh.K;
         break;
       case NK_ATTN:
         r.args.a.n_pages = sh.K;

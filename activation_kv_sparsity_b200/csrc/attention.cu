@@ -68,6 +68,16 @@ __global__ void __launch_bounds__(kAttnWarps * 32) k_attn(AttnArgs a) {
   const int g = lane >> 2, t = lane & 3;
   const int G = a.G;
 
+  // The cached pages do not depend on the previous kernel (it only appends
+  // to the last page, and L2 keeps that coherent): with the implicit page
+  // list, pull each warp's first two pages into L2 before waiting for it.
+  if (!a.pages && lane == 0) {
+    const int i0 = split * a.pages_per_split + warp;
+    const int i_end0 = min(a.n_pages, (split + 1) * a.pages_per_split);
+    for (int i = i0; i < i_end0 && i < i0 + 2 * kAttnWarps; i += kAttnWarps)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                   :: "l"(a.kv + ((size_t)h * a.Pmax + i) * PAGE_ELEMS), "r"(PAGE_ELEMS * 2) : "memory");
+  }
   pdl_wait();
   pdl_trigger();
 
@@ -279,8 +289,8 @@ void attn_plan(int n_pages, int Hkv, int sms, int* splits, int* pps) {
   const int target = 2 * sms;                   // two resident CTAs per SM (register bound)
   int s = std::max(1, (target + Hkv - 1) / Hkv);
   s = std::min(s, kMaxSplits);
-  // at least two pages per warp: short lists use fewer, fuller splits
-  s = std::min(s, std::max(1, n_pages / (2 * kAttnWarps)));
+  // at least one page per warp: short lists use fewer, fuller splits
+  s = std::min(s, std::max(1, n_pages / kAttnWarps));
   int per = (n_pages + s - 1) / s;
   per = std::max(per, 1);
   *pps = per;

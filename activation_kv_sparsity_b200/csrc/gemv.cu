@@ -42,6 +42,7 @@ namespace bc {
 constexpr int kGemvWarps = 8;
 constexpr int kGemvThreads = kGemvWarps * 32;
 constexpr int kRowsInFlight = 16;
+constexpr int kPrefetchRowsL2 = 512;   // dense rows per CTA pulled into L2 before the dependency wait
 
 __device__ __forceinline__ void fma8(float* acc, float xv, const uint4& w) {
   acc[0] = fmaf(xv, bf16_lo(w.x), acc[0]);
@@ -152,11 +153,16 @@ __global__ void __launch_bounds__(kGemvThreads, 2) k_gemv(GemvArgs a) {
   const size_t ld = (size_t)a.d_out;
   const int my0 = warp * RPI + lrow;              // this lane's first row in the run
 
-  // Weights do not depend on the previous kernel: in dense mode issue this
-  // lane's first batch of rows before waiting for it.
+  // Weights do not depend on the previous kernel: in dense mode pull the
+  // rows after the first batch into L2 and issue this lane's first batch of
+  // rows before waiting for it, so the stream overlaps the previous kernel's
+  // tail.
   uint4 w0[kRowsInFlight];
   bool first_loaded = false;
   if (!a.idx) {
+    for (int r = ROWS_STEP * kRowsInFlight + tid; r < min(nr, kPrefetchRowsL2); r += kGemvThreads)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                   :: "l"(a.W + (size_t)(r0 + r) * ld + col0), "r"(TW * 2) : "memory");
     #pragma unroll
     for (int u = 0; u < kRowsInFlight; ++u) {
       const int rr = my0 + u * ROWS_STEP;

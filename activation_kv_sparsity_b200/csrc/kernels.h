@@ -70,19 +70,19 @@ struct SelectArgs {
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl);
 
 // ------------------------------------------------------------------ KV pages
-// Page scores, then (by the last CTA of each kv head) the page select.
+// Page scores (grid-wide), then the page select (one cluster per kv head).
 struct PageArgs {
   const float* q;                 // rotated queries [Hkv*G][hd]
   const __nv_bfloat16* meta;      // layer key bounds [Hkv][Pmax][2][hd]
   int Hkv, G, hd, Pmax, P, K, sinks, recent;
   float* scores;                  // [Hkv][Pmax]
   int* pages;                     // [Hkv][Pmax], first K ascending
-  unsigned* counters;             // [Hkv], zero between launches
+  unsigned* counters;             // unused (kept for the workspace layout)
 };
-cudaError_t launch_pages(const PageArgs& a, cudaStream_t st, bool pdl);
-// Launch shape of the page kernel for P pages (graph node updates).
+cudaError_t launch_page_scores(const PageArgs& a, cudaStream_t st, bool pdl);
+cudaError_t launch_page_select(const PageArgs& a, cudaStream_t st, bool pdl);
+// Launch shape of the page scorer for P pages (graph node updates).
 dim3 pages_grid(const PageArgs& a);
-size_t pages_smem(const PageArgs& a);
 
 // ------------------------------------------------------------------ attention
 struct AttnArgs {

@@ -11,10 +11,9 @@
 //   the page key bound of Quest, listed among the paper's closest ancestors
 //   on its mlsanity page): s_p = max over the group's query heads of
 //   sum_c max(q_c*kmin_pc, q_c*kmax_pc).
-// * Page select, run by the last scoring CTA of each kv head to finish:
-//   forced sinks and recent pages plus the best-scored others (README, "What
-//   it does in one picture": sinks, part of the history and the recent
-//   entries).
+// * Page select, one cluster per kv head: forced sinks and recent pages plus
+//   the best-scored others (README, "What it does in one picture": sinks,
+//   part of the history and the recent entries).
 //
 // Exact top-k over 32-bit order keys: an interval search that splits the
 // candidates' key range into 256 bins per pass.  Only the first pass sweeps
@@ -25,6 +24,10 @@
 // ascending.
 #include "common.cuh"
 #include "kernels.h"
+
+#include <cooperative_groups.h>
+
+namespace cg = cooperative_groups;
 
 namespace bc {
 
@@ -202,22 +205,234 @@ __device__ void radix_topk(int n, int need, KeyF key, StateF state, int* out, To
 }
 
 // ------------------------------------------------------------------ activation select
-constexpr int kSelThreads2 = 1024;
+// Above 8192 elements a cluster of kSelCluster CTAs (one per SM) ranks one vector: CTA r owns the
+// r-th contiguous slice of it.  The key range, every pass's histogram and the
+// final placement offsets are combined through distributed shared memory
+// between hardware cluster barriers, so each CTA ends with the same cut and
+// writes the kept indices of its own slice at their global positions.
+constexpr int kSelCluster = 8;
+constexpr int kSelClThreads = 512;
+constexpr int kSelSlice = kMaxSelect / kSelCluster;   // largest slice
 
-__global__ void __launch_bounds__(kSelThreads2, 1) k_select(SelectArgs a) {
-  extern __shared__ __align__(16) uint32_t s_key[];
-  __shared__ TopkSmem<kSelThreads2> sm;
-  const int tid = threadIdx.x, n = a.n;
+struct SelClusterSmem {
+  int hist[2][256];
+  int ghist[256];
+  int red[32];
+  uint32_t rmin[32], rmax[32];
+  uint32_t lo, hi;
+  int gt_tot, eq_tot;
+  uint32_t bin;
+  int above, cnt;
+};
+
+// Ranks the candidates of a vector split over the cluster: this CTA holds the
+// keys of [s0, s0 + ns) in s_key, and lo/hi, the min and max candidate key it
+// saw.  Writes the forced elements and the `need` best candidates (ties to
+// the lower index) of the whole vector, ascending, to out.  Every CTA of the
+// cluster calls it with its slice; all threads of each CTA take part.
+template <typename StateF>
+__device__ void cluster_topk(const uint32_t* s_key, int s0, int ns, int need, StateF state, uint32_t lo,
+                             uint32_t hi, int* out, SelClusterSmem& sm, cg::cluster_group& cl) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    sm.rmin[warp] = lo;
+    sm.rmax[warp] = hi;
+  }
+  for (int b = tid; b < 2 * 256; b += kSelClThreads) (&sm.hist[0][0])[b] = 0;
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t l2 = 0xFFFFFFFFu, h2 = 0u;
+    for (int w = 0; w < kSelClThreads / 32; ++w) {
+      l2 = min(l2, sm.rmin[w]);
+      h2 = max(h2, sm.rmax[w]);
+    }
+    sm.lo = l2;
+    sm.hi = h2;
+  }
+  cl.sync();
+  lo = 0xFFFFFFFFu;
+  hi = 0u;
+  for (int q = 0; q < kSelCluster; ++q) {
+    lo = min(lo, *cl.map_shared_rank(&sm.lo, q));
+    hi = max(hi, *cl.map_shared_rank(&sm.hi, q));
+  }
+  uint32_t base = lo, span_m1 = hi - lo;
+  int rem = need;
+  if (need <= 0) span_m1 = 0;
+
+  // interval passes: local histograms of the slices, summed across the cluster
+  #pragma unroll 1
+  for (int pass = 0; pass < 5 && span_m1 > 0; ++pass) {
+    int* H = sm.hist[pass & 1];
+    const int sh = max(0, 24 - __clz(span_m1));
+    for (int j = tid; j < ns; j += kSelClThreads) {
+      if (state(s0 + j) != ST_CAND) continue;
+      const uint32_t kk = s_key[j];
+      if (kk >= base && kk - base <= span_m1) atomicAdd(&H[(kk - base) >> sh], 1);
+    }
+    cl.sync();   // every slice's histogram is complete; the other buffer is free
+    if (tid < 256) {
+      int g = 0;
+      #pragma unroll
+      for (int q = 0; q < kSelCluster; ++q) g += cl.map_shared_rank(H, q)[tid];
+      sm.ghist[tid] = g;
+      sm.hist[(pass + 1) & 1][tid] = 0;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int c[8], sum = 0;
+      #pragma unroll
+      for (int j = 0; j < 8; ++j) {              // lane owns bins 255-8*lane .. 248-8*lane
+        c[j] = sm.ghist[255 - 8 * lane - j];
+        sum += c[j];
+      }
+      int incl = sum;
+      #pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int above = incl - sum;
+      #pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (above < rem && above + c[j] >= rem) {
+          sm.bin = (uint32_t)(255 - 8 * lane - j);
+          sm.above = above;
+          sm.cnt = c[j];
+        }
+        above += c[j];
+      }
+    }
+    __syncthreads();
+    const uint32_t b_lo = sm.bin << sh;
+    rem -= sm.above;
+    const int cnt = sm.cnt;
+    base += b_lo;
+    span_m1 = min((1u << sh) - 1u, span_m1 - b_lo);
+    if (cnt == rem) break;                        // the whole bin is kept
+  }
+
+  // placement: forced elements, keys above the interval, and the first
+  // `rem` candidates (by index) inside it
+  const uint32_t top = base + span_m1;
+  const int per = (ns + kSelClThreads - 1) / kSelClThreads;
+  const int b0 = min(ns, tid * per), b1 = min(ns, b0 + per);
+  int gt = 0, eq = 0;
+  for (int j = b0; j < b1; ++j) {
+    const uint8_t st = state(s0 + j);
+    if (st == ST_FORCED) {
+      ++gt;
+    } else if (st == ST_CAND && need > 0) {
+      const uint32_t kk = s_key[j];
+      gt += kk > top;
+      eq += kk >= base && kk <= top;
+    }
+  }
+  int total;
+  const int excl = block_excl_scan<kSelClThreads>((gt << 16) | eq, sm.red, &total);
+  if (tid == 0) {
+    sm.gt_tot = total >> 16;
+    sm.eq_tot = total & 0xFFFF;
+  }
+  cl.sync();
+  int gt_before = 0, eq_before = 0;
+  for (int q = 0; q < (int)cl.block_rank(); ++q) {
+    gt_before += *cl.map_shared_rank(&sm.gt_tot, q);
+    eq_before += *cl.map_shared_rank(&sm.eq_tot, q);
+  }
+  int er = eq_before + (excl & 0xFFFF);
+  int pos = gt_before + (excl >> 16) + min(er, rem);
+  for (int j = b0; j < b1; ++j) {
+    const uint8_t st = state(s0 + j);
+    bool keep = st == ST_FORCED;
+    if (st == ST_CAND && need > 0) {
+      const uint32_t kk = s_key[j];
+      if (kk > top) {
+        keep = true;
+      } else if (kk >= base) {
+        keep = er < rem;
+        ++er;
+      }
+    }
+    if (keep) out[pos++] = s0 + j;
+  }
+  cl.sync();   // peers may still be reading this CTA's totals
+}
+
+__global__ void __launch_bounds__(kSelClThreads, 1) k_select(SelectArgs a) {
+  __shared__ uint32_t s_key[kSelSlice];
+  __shared__ SelClusterSmem sm;
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = (int)cl.block_rank();
+  const int tid = threadIdx.x;
+  const int n = a.n;
+  const int s0 = (int)(((long long)n * rank) / kSelCluster);
+  const int ns = (int)(((long long)n * (rank + 1)) / kSelCluster) - s0;
   pdl_wait();
   pdl_trigger();
-  // prep: 8 elements per thread per round, their loads in flight together
+
+  // the slice's keys, with 8 elements per thread per round of loads
   uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  for (int j = tid; j < 256; j += kSelThreads2) sm.hist[j] = 0;
-  for (int i0 = 0; i0 < n; i0 += 8 * kSelThreads2) {
+  for (int j0 = 0; j0 < ns; j0 += 8 * kSelClThreads) {
     float a0[8], a1[8];
     #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kSelThreads2 + tid;
+      const int j = j0 + u * kSelClThreads + tid, i = s0 + j;
+      a0[u] = 0.f;
+      a1[u] = 0.f;
+      if (j < ns) {
+        switch (a.prep) {
+          case SP_NORM: a0[u] = a.x[i]; a1[u] = bf16f(a.gain[i]); break;
+          case SP_EMBED_NORM: a0[u] = bf16f(a.embed_row[i]); a1[u] = bf16f(a.gain[i]); break;
+          case SP_SWIGLU: a0[u] = a.x[i]; a1[u] = a.x[n + i]; break;
+          default: a0[u] = a.x[i];
+        }
+      }
+    }
+    #pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * kSelClThreads + tid, i = s0 + j;
+      if (j >= ns) break;
+      float v;
+      switch (a.prep) {
+        case SP_NORM: v = a0[u] * a1[u]; break;
+        case SP_EMBED_NORM: a.x_init[i] = a0[u]; v = a0[u] * a1[u]; break;
+        case SP_SWIGLU: v = a0[u] / (1.0f + expf(-a0[u])) * a1[u]; break;
+        default: v = a0[u];
+      }
+      if (a.vout) a.vout[i] = v;
+      const uint32_t kk = __float_as_uint(fabsf(v));
+      s_key[j] = kk;
+      lo = min(lo, kk);
+      hi = max(hi, kk);
+    }
+  }
+  cluster_topk(s_key, s0, ns, a.k, [](int) { return (uint8_t)ST_CAND; }, lo, hi, a.idx, sm, cl);
+}
+
+// Vectors up to kSelOneCta elements: one CTA ranks the whole vector (a
+// cluster's barriers cost more than they save at this size).
+constexpr int kSelOneCta = 8192;
+constexpr int kSelThreads1 = 1024;
+
+__global__ void __launch_bounds__(kSelThreads1, 1) k_select_cta(SelectArgs a) {
+  __shared__ uint32_t s_key[kSelOneCta];
+  __shared__ TopkSmem<kSelThreads1> sm;
+  const int tid = threadIdx.x, n = a.n;
+  pdl_wait();
+  pdl_trigger();
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (int j = tid; j < 256; j += kSelThreads1) sm.hist[j] = 0;
+  for (int i0 = 0; i0 < n; i0 += 8 * kSelThreads1) {
+    float a0[8], a1[8];
+    #pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kSelThreads1 + tid;
       a0[u] = 0.f;
       a1[u] = 0.f;
       if (i < n) {
@@ -231,7 +446,7 @@ __global__ void __launch_bounds__(kSelThreads2, 1) k_select(SelectArgs a) {
     }
     #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kSelThreads2 + tid;
+      const int i = i0 + u * kSelThreads1 + tid;
       if (i >= n) break;
       float v;
       switch (a.prep) {
@@ -248,28 +463,35 @@ __global__ void __launch_bounds__(kSelThreads2, 1) k_select(SelectArgs a) {
     }
   }
   __syncthreads();
-  radix_topk<kSelThreads2>(
+  radix_topk<kSelThreads1>(
       n, a.k, [&](int i) { return s_key[i]; }, [](int) { return (uint8_t)ST_CAND; }, a.idx, sm, lo, hi);
 }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl) {
-  const size_t smem = (size_t)kMaxSelect * sizeof(uint32_t);
-  static bool attr_done = false;
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(1);
-  cfg.blockDim = dim3(kSelThreads2);
-  cfg.dynamicSmemBytes = (size_t)a.n * sizeof(uint32_t);
+  if (a.n <= kSelOneCta) {
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(kSelThreads1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr1[1];
+    attr1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr1[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr1;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_select_cta, a);
+  }
+  cfg.gridDim = dim3(kSelCluster);
+  cfg.blockDim = dim3(kSelClThreads);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kSelCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, k_select, a);
 }
 
@@ -283,8 +505,6 @@ __global__ void __launch_bounds__(kPageThreads) k_pages(PageArgs a) {
   constexpr int LPP = HD / 8;          // lanes per page
   constexpr int PPW = 32 / LPP;        // pages per warp step
   constexpr int PAGES_PER_CTA = (kPageThreads / 32) * PPW * 4;
-  __shared__ TopkSmem<kPageThreads> sm;
-  __shared__ int s_last;
   const int h = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int sub = lane / LPP, cl = lane % LPP;
@@ -292,25 +512,39 @@ __global__ void __launch_bounds__(kPageThreads) k_pages(PageArgs a) {
   pdl_trigger();
   float qv[8][8];   // [head][channel], G <= 8
   #pragma unroll
-  for (int g = 0; g < 8; ++g)
-    #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      qv[g][j] = (g < a.G) ? a.q[(size_t)(h * a.G + g) * HD + cl * 8 + j] : 0.f;
+  for (int g = 0; g < 8; ++g) {
+    float4 q0 = make_float4(0.f, 0.f, 0.f, 0.f), q1 = q0;
+    if (g < a.G) {
+      const float4* qp = reinterpret_cast<const float4*>(a.q + (size_t)(h * a.G + g) * HD + cl * 8);
+      q0 = qp[0];
+      q1 = qp[1];
+    }
+    qv[g][0] = q0.x; qv[g][1] = q0.y; qv[g][2] = q0.z; qv[g][3] = q0.w;
+    qv[g][4] = q1.x; qv[g][5] = q1.y; qv[g][6] = q1.z; qv[g][7] = q1.w;
+  }
   const int p_begin = blockIdx.x * PAGES_PER_CTA;
   const int p_end = min(a.P, p_begin + PAGES_PER_CTA);
   const __nv_bfloat16* mbase = a.meta + (size_t)h * a.Pmax * 2 * HD;
   float* scores = a.scores + (size_t)h * a.Pmax;
-  // warp-uniform loop: every lane takes part in the shuffles
-  for (int pb = p_begin + warp * PPW; pb < p_end; pb += (kPageThreads / 32) * PPW) {
-    const int p = pb + sub;
-    const bool valid = p < p_end;
-    uint4 mn = make_uint4(0, 0, 0, 0), mx = make_uint4(0, 0, 0, 0);
-    if (valid) {
+  // all of this lane's bounds in one round of loads (4 steps of the warp)
+  constexpr int STEPS = PAGES_PER_CTA / ((kPageThreads / 32) * PPW);
+  uint4 mn[STEPS], mx[STEPS];
+  #pragma unroll
+  for (int it = 0; it < STEPS; ++it) {
+    const int p = p_begin + (it * (kPageThreads / 32) + warp) * PPW + sub;
+    mn[it] = make_uint4(0, 0, 0, 0);
+    mx[it] = mn[it];
+    if (p < p_end) {
       const __nv_bfloat16* mp = mbase + (size_t)p * 2 * HD + cl * 8;
-      mn = ld_stream(mp);
-      mx = ld_stream(mp + HD);
+      mn[it] = ld_stream(mp);
+      mx[it] = ld_stream(mp + HD);
     }
-    const uint32_t mnw[4] = {mn.x, mn.y, mn.z, mn.w}, mxw[4] = {mx.x, mx.y, mx.z, mx.w};
+  }
+  #pragma unroll
+  for (int it = 0; it < STEPS; ++it) {
+    const int p = p_begin + (it * (kPageThreads / 32) + warp) * PPW + sub;
+    const uint32_t mnw[4] = {mn[it].x, mn[it].y, mn[it].z, mn[it].w};
+    const uint32_t mxw[4] = {mx[it].x, mx[it].y, mx[it].z, mx[it].w};
     float best = -INFINITY;
     #pragma unroll
     for (int g = 0; g < 8; ++g) {
@@ -327,36 +561,41 @@ __global__ void __launch_bounds__(kPageThreads) k_pages(PageArgs a) {
       for (int o = LPP / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o, LPP);
       best = fmaxf(best, s);
     }
-    if (valid && cl == 0) scores[p] = best;
+    if (p < p_end && cl == 0) scores[p] = best;
   }
-  // the last CTA of this kv head to finish selects its pages
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&a.counters[h], 1u) == gridDim.x - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  if (tid == 0) a.counters[h] = 0u;
+}
+
+// Page select: one cluster per kv head; CTA r ranks the r-th slice of the
+// head's page scores.  Forced pages (sinks, recent) are kept and not ranked.
+__global__ void __launch_bounds__(kSelClThreads, 1) k_page_select(PageArgs a) {
+  __shared__ uint32_t s_key[kSelSlice];
+  __shared__ SelClusterSmem sm;
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = (int)cl.block_rank();
+  const int h = blockIdx.y, tid = threadIdx.x;
   const int P = a.P;
-  extern __shared__ __align__(16) uint32_t s_key[];
+  const int s0 = (int)(((long long)P * rank) / kSelCluster);
+  const int ns = (int)(((long long)P * (rank + 1)) / kSelCluster) - s0;
+  pdl_wait();
+  pdl_trigger();
   const int sink_end = min(a.sinks, P), rec_begin = max(P - a.recent, 0);
   const int n_forced = sink_end + (P - max(rec_begin, sink_end));
+  const float* scores = a.scores + (size_t)h * a.Pmax;
   uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  for (int j = tid; j < 256; j += kPageThreads) sm.hist[j] = 0;
-  #pragma unroll 8
-  for (int i = tid; i < P; i += kPageThreads) {
-    const uint32_t kk = float_order_key(ld_cg(&scores[i]));
-    s_key[i] = kk;
+  #pragma unroll 4
+  for (int j = tid; j < ns; j += kSelClThreads) {
+    const int i = s0 + j;
+    const uint32_t kk = float_order_key(scores[i]);
+    s_key[j] = kk;
     if (i >= sink_end && i < rec_begin) {
       lo = min(lo, kk);
       hi = max(hi, kk);
     }
   }
-  __syncthreads();
-  radix_topk<kPageThreads>(
-      P, a.K - n_forced, [&](int i) { return s_key[i]; },
-      [&](int i) { return (uint8_t)((i < sink_end || i >= rec_begin) ? ST_FORCED : ST_CAND); },
-      a.pages + (size_t)h * a.Pmax, sm, lo, hi);
+  cluster_topk(
+      s_key, s0, ns, a.K - n_forced,
+      [&](int i) { return (uint8_t)((i < sink_end || i >= rec_begin) ? ST_FORCED : ST_CAND); }, lo, hi,
+      a.pages + (size_t)h * a.Pmax, sm, cl);
 }
 
 dim3 pages_grid(const PageArgs& a) {
@@ -364,23 +603,13 @@ dim3 pages_grid(const PageArgs& a) {
   return dim3((a.P + ppc - 1) / ppc, a.Hkv);
 }
 
-size_t pages_smem(const PageArgs& a) { return (size_t)a.P * sizeof(uint32_t); }
 
-cudaError_t launch_pages(const PageArgs& a, cudaStream_t st, bool pdl) {
-  static bool attr_done = false;
-  if (!attr_done) {
-    const int smem = kMaxSelect * (int)sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(k_pages<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_pages<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
+cudaError_t launch_page_scores(const PageArgs& a, cudaStream_t st, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = pages_grid(a);
   cfg.blockDim = dim3(kPageThreads);
-  cfg.dynamicSmemBytes = pages_smem(a);
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
@@ -388,6 +617,23 @@ cudaError_t launch_pages(const PageArgs& a, cudaStream_t st, bool pdl) {
   if (a.hd == 128) return cudaLaunchKernelEx(&cfg, k_pages<128>, a);
   if (a.hd == 64) return cudaLaunchKernelEx(&cfg, k_pages<64>, a);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_page_select(const PageArgs& a, cudaStream_t st, bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kSelCluster, a.Hkv);
+  cfg.blockDim = dim3(kSelClThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kSelCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, k_page_select, a);
 }
 
 }  // namespace bc
