@@ -13,11 +13,12 @@
 // G <= 8 query heads of the group rounded to bf16 ("hi"), rows 8..15 the
 // rounding residues ("lo"), so S = S_hi + S_lo keeps about 16 significant
 // bits of the fp32 query; the softmax weights P are split the same way for
-// P*V.  Keys are loaded straight into B fragments: lane (g, t) reads 32
-// consecutive dims of key rows g and g+8, and the contraction dims are
-// permuted consistently in A and B, which leaves the dot products unchanged.
-// Value fragments are transposed in registers with movmatrix.  Each lane
-// ends with its head row's output over hd/4 consecutive dims.
+// P*V.  Keys are loaded straight into B fragments: lane (g, t) reads dims
+// u*32 + t*8 .. +8 (u = 0..hd/32-1) of key rows g and g+8, so the four lanes
+// of a row read 64 contiguous bytes per instruction, and the contraction
+// dims are permuted consistently in A and B, which leaves the dot products
+// unchanged.  Value fragments are transposed in registers with movmatrix;
+// each lane ends with its head row's output over the same dims.
 //
 // Partials (m, l, o) per (query head, split) use base-2 logits.  The last
 // CTA of each kv head to finish (an atomic ticket, no spinning) merges them:
@@ -53,7 +54,7 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
 }
 
 template <int HD>
-__global__ void __launch_bounds__(kAttnWarps * 32) k_attn(AttnArgs a) {
+__global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn(AttnArgs a) {
   constexpr int KSTEPS = HD / 16;   // k16 steps of q.k
   constexpr int NBLK = HD / 8;      // n8 blocks of p.v
   constexpr int DPL = HD / 4;       // dims per lane
@@ -85,15 +86,17 @@ __global__ void __launch_bounds__(kAttnWarps * 32) k_attn(AttnArgs a) {
   const float qscale = 1.4426950408889634f * rsqrtf((float)HD);
   uint32_t qa[KSTEPS][4];
   {
-    const float* qrow = a.q + (size_t)(h * G + g) * HD + t * DPL;
+    const float* qrow = a.q + (size_t)(h * G + g) * HD + t * 8;
     #pragma unroll
     for (int s = 0; s < KSTEPS; ++s) {
+      // k-step s contracts dims (s/2)*32 + t*8 + 4*(s%2) + 0..3 of this lane
+      const int d0 = (s / 2) * 32 + 4 * (s % 2);
       float q0 = 0.f, q1 = 0.f, q2 = 0.f, q3 = 0.f;
       if (g < G) {
-        q0 = qrow[4 * s] * qscale;
-        q1 = qrow[4 * s + 1] * qscale;
-        q2 = qrow[4 * s + 2] * qscale;
-        q3 = qrow[4 * s + 3] * qscale;
+        q0 = qrow[d0] * qscale;
+        q1 = qrow[d0 + 1] * qscale;
+        q2 = qrow[d0 + 2] * qscale;
+        q3 = qrow[d0 + 3] * qscale;
       }
       split2(q0, q1, qa[s][0], qa[s][1]);
       split2(q2, q3, qa[s][2], qa[s][3]);
@@ -110,24 +113,22 @@ __global__ void __launch_bounds__(kAttnWarps * 32) k_attn(AttnArgs a) {
   const __nv_bfloat16* head_base = a.kv + (size_t)h * a.Pmax * PAGE_ELEMS;
   const int* plist = a.pages ? a.pages + (size_t)h * a.Pmax : nullptr;
 
-  for (int i = i_begin + warp; i < i_end; i += kAttnWarps) {
-    const int page = plist ? plist[i] : i;
-    const int nxt = i + kAttnWarps;
-    if (lane == 0 && nxt < i_end) {
-      const int pn = plist ? plist[nxt] : nxt;
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
-                   :: "l"(head_base + (size_t)pn * PAGE_ELEMS), "r"(PAGE_ELEMS * 2) : "memory");
-    }
-    const __nv_bfloat16* pk = head_base + (size_t)page * PAGE_ELEMS + t * DPL;
+  // one page: keys then values of 16 tokens, lane (g, t) holds 32 dims of
+  // token rows g and g+8
+  // lane (g, t) takes dims u*32 + t*8 .. +8 of its rows: the four lanes of a
+  // row cover 64 contiguous bytes per load, whole 32-byte sectors
+  auto load_page = [&](int page, uint4* k0, uint4* k1, uint4* v0, uint4* v1) {
+    const __nv_bfloat16* pk = head_base + (size_t)page * PAGE_ELEMS + t * 8;
     const __nv_bfloat16* pv = pk + kPage * HD;
-    uint4 k0[U4], k1[U4], v0[U4], v1[U4];
     #pragma unroll
     for (int u = 0; u < U4; ++u) {
-      k0[u] = ld_stream(pk + g * HD + 8 * u);
-      k1[u] = ld_stream(pk + (g + 8) * HD + 8 * u);
-      v0[u] = ld_stream(pv + g * HD + 8 * u);
-      v1[u] = ld_stream(pv + (g + 8) * HD + 8 * u);
+      k0[u] = ld_stream(pk + g * HD + 32 * u);
+      k1[u] = ld_stream(pk + (g + 8) * HD + 32 * u);
+      v0[u] = ld_stream(pv + g * HD + 32 * u);
+      v1[u] = ld_stream(pv + (g + 8) * HD + 32 * u);
     }
+  };
+  auto process_page = [&](int page, uint4* k0, uint4* k1, uint4* v0, uint4* v1) {
     const int valid = min(kPage, a.n_tok - page * kPage);
     if (g >= valid) {
       #pragma unroll
@@ -177,6 +178,32 @@ __global__ void __launch_bounds__(kAttnWarps * 32) k_attn(AttnArgs a) {
       const uint32_t b1 = transpose8x8(vr1[b]);
       mma16816(o[b], pa, b0, b1);
     }
+  };
+  auto page_at = [&](int i) { return plist ? plist[i] : i; };
+  auto prefetch = [&](int i) {
+    if (lane == 0 && i < i_end)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                   :: "l"(head_base + (size_t)page_at(i) * PAGE_ELEMS), "r"(PAGE_ELEMS * 2) : "memory");
+  };
+
+  // ping-pong over two register buffers: the next page is in flight while
+  // this one is processed, and pages two steps ahead are pulled into L2
+  uint4 ka0[U4], ka1[U4], va0[U4], va1[U4];
+  uint4 kb0[U4], kb1[U4], vb0[U4], vb1[U4];
+  int i = i_begin + warp;
+  if (i < i_end) load_page(page_at(i), ka0, ka1, va0, va1);
+  while (i < i_end) {
+    int j = i + kAttnWarps;
+    prefetch(j + kAttnWarps);
+    if (j < i_end) load_page(page_at(j), kb0, kb1, vb0, vb1);
+    process_page(page_at(i), ka0, ka1, va0, va1);
+    i = j;
+    if (i >= i_end) break;
+    j = i + kAttnWarps;
+    prefetch(j + kAttnWarps);
+    if (j < i_end) load_page(page_at(j), ka0, ka1, va0, va1);
+    process_page(page_at(i), kb0, kb1, vb0, vb1);
+    i = j;
   }
 
   // this warp's state for head row g (lanes of a quad share it)
@@ -184,9 +211,10 @@ __global__ void __launch_bounds__(kAttnWarps * 32) k_attn(AttnArgs a) {
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
   if (g < G) {
     #pragma unroll
-    for (int b = 0; b < NBLK; ++b) {
-      s_o[warp][g][t * DPL + 2 * b] = o[b][0] + o[b][2];
-      s_o[warp][g][t * DPL + 2 * b + 1] = o[b][1] + o[b][3];
+    for (int b = 0; b < NBLK; ++b) {         // block b holds dims (b/4)*32 + t*8 + 2*(b%4) + 0..1
+      const int dd = (b / 4) * 32 + t * 8 + 2 * (b % 4);
+      s_o[warp][g][dd] = o[b][0] + o[b][2];
+      s_o[warp][g][dd + 1] = o[b][1] + o[b][3];
     }
     if (t == 0) {
       s_m[warp][g] = m_run;
