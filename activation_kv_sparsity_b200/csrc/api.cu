@@ -521,7 +521,8 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
     if (!record(rec, st, NK_QKV, l, ga)) return fail(BC_ECUDA, "capture: no node");
     ++launches;
     if (kvs) {
-      PageArgs pa{q, metal, Hkv, G, hd, Pmax, P, K, sinks, recent, pscore, pages, page_counters};
+      PageArgs pa{q, metal, Hkv, G, hd, Pmax, P, K, sinks, recent, page_rounds(P, hd, Hkv, m->sms),
+                  pscore, pages, page_counters};
       BC_CUDA(launch_page_scores(pa, st, true), "page scores");
       if (!record(rec, st, NK_PAGES, l, pa)) return fail(BC_ECUDA, "capture: no node");
       BC_CUDA(launch_page_select(pa, st, true), "page select");
@@ -637,6 +638,7 @@ static cudaError_t launch_step_graph(bc_model* m, StepGraph* g, int token, const
       case NK_PAGES:
         r.args.p.P = sh.P;
         r.args.p.K = sh.K;
+        r.args.p.rounds = page_rounds(sh.P, c.head_dim, c.n_kv_heads, m->sms);
         kp.gridDim = pages_grid(r.args.p);
         break;
       case NK_PAGE_SEL:

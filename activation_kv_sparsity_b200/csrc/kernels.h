@@ -75,6 +75,7 @@ struct PageArgs {
   const float* q;                 // rotated queries [Hkv*G][hd]
   const __nv_bfloat16* meta;      // layer key bounds [Hkv][Pmax][2][hd]
   int Hkv, G, hd, Pmax, P, K, sinks, recent;
+  int rounds;                     // scorer: rounds of pages per CTA (page_rounds)
   float* scores;                  // [Hkv][Pmax]
   int* pages;                     // [Hkv][Pmax], first K ascending
   unsigned* counters;             // unused (kept for the workspace layout)
@@ -82,6 +83,7 @@ struct PageArgs {
 cudaError_t launch_page_scores(const PageArgs& a, cudaStream_t st, bool pdl);
 cudaError_t launch_page_select(const PageArgs& a, cudaStream_t st, bool pdl);
 // Launch shape of the page scorer for P pages (graph node updates).
+int page_rounds(int P, int hd, int Hkv, int sms);
 dim3 pages_grid(const PageArgs& a);
 
 // ------------------------------------------------------------------ attention

@@ -497,22 +497,30 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl) {
 
 // ------------------------------------------------------------------ page scores + select
 // A group of hd/8 lanes scores one page: each lane holds 8 channels of the
-// group's G queries and reads 16 bytes of kmin and 16 bytes of kmax.
+// group's queries and reads 16 bytes of kmin and 16 bytes of kmax.  A CTA
+// walks `rounds` rounds of 64 pages (at hd = 128); the next round's bounds
+// are in flight while the current round is scored.
 constexpr int kPageThreads = 256;
 
 template <int HD>
-__global__ void __launch_bounds__(kPageThreads) k_pages(PageArgs a) {
+__host__ __device__ constexpr int pages_per_round() {
+  return (kPageThreads / 32) * (32 / (HD / 8)) * 4;
+}
+
+template <int HD, int GMAX>
+__global__ void __launch_bounds__(kPageThreads, GMAX <= 4 ? 2 : 1) k_pages(PageArgs a) {
   constexpr int LPP = HD / 8;          // lanes per page
   constexpr int PPW = 32 / LPP;        // pages per warp step
-  constexpr int PAGES_PER_CTA = (kPageThreads / 32) * PPW * 4;
+  constexpr int STEPS = 4;             // warp steps per round
+  constexpr int PPR = pages_per_round<HD>();
   const int h = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int sub = lane / LPP, cl = lane % LPP;
   pdl_wait();
   pdl_trigger();
-  float qv[8][8];   // [head][channel], G <= 8
+  float qv[GMAX][8];   // [head][channel]
   #pragma unroll
-  for (int g = 0; g < 8; ++g) {
+  for (int g = 0; g < GMAX; ++g) {
     float4 q0 = make_float4(0.f, 0.f, 0.f, 0.f), q1 = q0;
     if (g < a.G) {
       const float4* qp = reinterpret_cast<const float4*>(a.q + (size_t)(h * a.G + g) * HD + cl * 8);
@@ -522,46 +530,56 @@ __global__ void __launch_bounds__(kPageThreads) k_pages(PageArgs a) {
     qv[g][0] = q0.x; qv[g][1] = q0.y; qv[g][2] = q0.z; qv[g][3] = q0.w;
     qv[g][4] = q1.x; qv[g][5] = q1.y; qv[g][6] = q1.z; qv[g][7] = q1.w;
   }
-  const int p_begin = blockIdx.x * PAGES_PER_CTA;
-  const int p_end = min(a.P, p_begin + PAGES_PER_CTA);
   const __nv_bfloat16* mbase = a.meta + (size_t)h * a.Pmax * 2 * HD;
   float* scores = a.scores + (size_t)h * a.Pmax;
-  // all of this lane's bounds in one round of loads (4 steps of the warp)
-  constexpr int STEPS = PAGES_PER_CTA / ((kPageThreads / 32) * PPW);
-  uint4 mn[STEPS], mx[STEPS];
-  #pragma unroll
-  for (int it = 0; it < STEPS; ++it) {
-    const int p = p_begin + (it * (kPageThreads / 32) + warp) * PPW + sub;
-    mn[it] = make_uint4(0, 0, 0, 0);
-    mx[it] = mn[it];
-    if (p < p_end) {
-      const __nv_bfloat16* mp = mbase + (size_t)p * 2 * HD + cl * 8;
-      mn[it] = ld_stream(mp);
-      mx[it] = ld_stream(mp + HD);
-    }
-  }
-  #pragma unroll
-  for (int it = 0; it < STEPS; ++it) {
-    const int p = p_begin + (it * (kPageThreads / 32) + warp) * PPW + sub;
-    const uint32_t mnw[4] = {mn[it].x, mn[it].y, mn[it].z, mn[it].w};
-    const uint32_t mxw[4] = {mx[it].x, mx[it].y, mx[it].z, mx[it].w};
-    float best = -INFINITY;
+  const int p_cta = blockIdx.x * a.rounds * PPR;
+  auto page_of = [&](int round, int it) { return p_cta + round * PPR + (it * (kPageThreads / 32) + warp) * PPW + sub; };
+  auto load_round = [&](int round, uint4* mn, uint4* mx) {
     #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      if (g >= a.G) break;
-      float s = 0.f;
-      #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float lo0 = bf16_lo(mnw[j]), lo1 = bf16_hi(mnw[j]);
-        const float hi0 = bf16_lo(mxw[j]), hi1 = bf16_hi(mxw[j]);
-        s += fmaxf(qv[g][2 * j] * lo0, qv[g][2 * j] * hi0);
-        s += fmaxf(qv[g][2 * j + 1] * lo1, qv[g][2 * j + 1] * hi1);
+    for (int it = 0; it < STEPS; ++it) {
+      const int p = page_of(round, it);
+      mn[it] = make_uint4(0, 0, 0, 0);
+      mx[it] = mn[it];
+      if (round < a.rounds && p < a.P) {
+        const __nv_bfloat16* mp = mbase + (size_t)p * 2 * HD + cl * 8;
+        mn[it] = ld_stream(mp);
+        mx[it] = ld_stream(mp + HD);
       }
-      #pragma unroll
-      for (int o = LPP / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o, LPP);
-      best = fmaxf(best, s);
     }
-    if (p < p_end && cl == 0) scores[p] = best;
+  };
+  auto score_round = [&](int round, const uint4* mn, const uint4* mx) {
+    #pragma unroll
+    for (int it = 0; it < STEPS; ++it) {
+      const int p = page_of(round, it);
+      const uint32_t mnw[4] = {mn[it].x, mn[it].y, mn[it].z, mn[it].w};
+      const uint32_t mxw[4] = {mx[it].x, mx[it].y, mx[it].z, mx[it].w};
+      float best = -INFINITY;
+      #pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        if (g >= a.G) break;
+        float s = 0.f;
+        #pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float lo0 = bf16_lo(mnw[j]), lo1 = bf16_hi(mnw[j]);
+          const float hi0 = bf16_lo(mxw[j]), hi1 = bf16_hi(mxw[j]);
+          s += fmaxf(qv[g][2 * j] * lo0, qv[g][2 * j] * hi0);
+          s += fmaxf(qv[g][2 * j + 1] * lo1, qv[g][2 * j + 1] * hi1);
+        }
+        #pragma unroll
+        for (int o = LPP / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o, LPP);
+        best = fmaxf(best, s);
+      }
+      if (p < a.P && cl == 0) scores[p] = best;
+    }
+  };
+  uint4 mna[STEPS], mxa[STEPS], mnb[STEPS], mxb[STEPS];
+  load_round(0, mna, mxa);
+  for (int r = 0; r < a.rounds; r += 2) {
+    load_round(r + 1, mnb, mxb);
+    score_round(r, mna, mxa);
+    if (r + 1 >= a.rounds) break;
+    load_round(r + 2, mna, mxa);
+    score_round(r + 1, mnb, mxb);
   }
 }
 
@@ -598,24 +616,31 @@ __global__ void __launch_bounds__(kSelClThreads, 1) k_page_select(PageArgs a) {
       a.pages + (size_t)h * a.Pmax, sm, cl);
 }
 
-dim3 pages_grid(const PageArgs& a) {
-  const int ppc = (kPageThreads / 32) * (32 / (a.hd / 8)) * 4;
-  return dim3((a.P + ppc - 1) / ppc, a.Hkv);
+int page_rounds(int P, int hd, int Hkv, int sms) {
+  const int ppr = hd == 128 ? pages_per_round<128>() : pages_per_round<64>();
+  const int units = Hkv * ((P + ppr - 1) / ppr);          // rounds of work in all
+  const int r = (units + 2 * sms - 1) / (2 * sms);        // about two CTAs per SM
+  return r < 1 ? 1 : (r > 8 ? 8 : r);
 }
 
+dim3 pages_grid(const PageArgs& a) {
+  const int ppc = (a.hd == 128 ? pages_per_round<128>() : pages_per_round<64>()) * a.rounds;
+  return dim3((a.P + ppc - 1) / ppc, a.Hkv);
+}
 
 cudaError_t launch_page_scores(const PageArgs& a, cudaStream_t st, bool pdl) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = pages_grid(a);
   cfg.blockDim = dim3(kPageThreads);
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  if (a.hd == 128) return cudaLaunchKernelEx(&cfg, k_pages<128>, a);
-  if (a.hd == 64) return cudaLaunchKernelEx(&cfg, k_pages<64>, a);
+  const bool g4 = a.G <= 4;
+  if (a.hd == 128) return g4 ? cudaLaunchKernelEx(&cfg, k_pages<128, 4>, a) : cudaLaunchKernelEx(&cfg, k_pages<128, 8>, a);
+  if (a.hd == 64) return g4 ? cudaLaunchKernelEx(&cfg, k_pages<64, 4>, a) : cudaLaunchKernelEx(&cfg, k_pages<64, 8>, a);
   return cudaErrorInvalidValue;
 }
 
