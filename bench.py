@@ -284,12 +284,15 @@ def run_ours(args, rank, ws, local):
     attn = None
 
     clk = clocks.summary()
-    # measured crossings against the byte-account n*
+    # measured crossing against the byte account: the paper form (Equation 5)
+    # and this implementation's bytes (which add the page bounds the scorer reads)
     crossings = {}
     for rp, rkv in CROSS_PAIRS:
         acc = bc.byte_account(cfg, "both", 1024, rp=rp, rkv=rkv)
-        crossings[f"{rp}/{rkv}"] = {"n_star_tokens": round(acc["n_star"], 1)}
+        crossings[f"{rp}/{rkv}"] = {"n_star_tokens": round(acc["n_star"], 1),
+                                    "n_star_impl_tokens": impl_crossing(bc, cfg, rp, rkv)}
     cross_measured = measured_crossing(cells, contexts)
+    cross_measured["cost_aware_prediction"] = cost_aware_prediction(cells, contexts, cfg, bc)
 
     result = {
         "metric": METRIC,
@@ -327,6 +330,64 @@ def run_ours(args, rank, ws, local):
     return result
 
 
+def impl_crossing(bc, cfg, rp, rkv, sinks=1, recent=16):
+    """Context at which the act and kv steps of this library move the same
+    bytes (bc_byte_account's implementation form), by bisection."""
+    def diff(n):
+        a = bc.byte_account(cfg, "act", n, rp=rp, sinks=sinks, recent=recent)["impl_total_bytes"]
+        k = bc.byte_account(cfg, "kv", n, rkv=rkv, sinks=sinks, recent=recent)["impl_total_bytes"]
+        return a - k          # negative while the projection branch moves fewer bytes
+    lo, hi = 1, 1 << 21
+    if diff(lo) >= 0 or diff(hi) <= 0:
+        return None
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        if diff(mid) < 0:
+            lo = mid
+        else:
+            hi = mid
+    return hi
+
+
+def cost_aware_prediction(cells, contexts, cfg, bc):
+    """The pages' cost-aware prediction restated for this library: per mode,
+    step time = byte-account bytes / B + c (one bandwidth B for all modes,
+    one fixed per-step kernel cost c per mode), fitted by least squares over
+    the sampled contexts; the predicted crossing is where the act and kv fits
+    meet.  Returns the fit and the predicted crossing in tokens."""
+    import numpy as np
+    modes = [m for m in ("dense", "act", "kv") if all((m, n) in cells for n in contexts)]
+    if len(modes) < 3:
+        return None
+    rows, ys = [], []
+    for j, m in enumerate(modes):
+        for n in contexts:
+            c = cells[(m, n)]
+            r = [c["bytes_per_step"] / 1e9] + [1.0 if k == j else 0.0 for k in range(len(modes))]
+            rows.append(r)
+            ys.append(c["ms_per_step"] * 1e-3)
+    sol, *_ = np.linalg.lstsq(np.array(rows), np.array(ys), rcond=None)
+    inv_bw, costs = sol[0], dict(zip(modes, sol[1:]))
+    kw = dict(KEEP)
+
+    def t(mode, n):
+        return bc.byte_account(cfg, mode, n, **kw)["impl_total_bytes"] / 1e9 * inv_bw + costs[mode]
+    lo, hi = 1, 1 << 21
+    if (t("act", lo) - t("kv", lo)) * (t("act", hi) - t("kv", hi)) > 0:
+        pred = None
+    else:
+        while hi - lo > 1:
+            mid = (lo + hi) // 2
+            if t("act", mid) < t("kv", mid):
+                lo = mid
+            else:
+                hi = mid
+        pred = hi
+    return {"fit_gbs": round(1.0 / inv_bw, 1),
+            "fixed_cost_ms": {m: round(v * 1e3, 4) for m, v in costs.items()},
+            "predicted_act_vs_kv_tokens": pred}
+
+
 def measured_crossing(cells, contexts):
     """Context where the KV branch starts to beat the projection branch,
     interpolated linearly between the sampled contexts (the README's
@@ -337,7 +398,8 @@ def measured_crossing(cells, contexts):
     diff = [(n, cells[("act", n)]["ms_per_step"] - cells[("kv", n)]["ms_per_step"]) for n in ctx]
     for (n0, d0), (n1, d1) in zip(diff, diff[1:]):
         if d0 < 0 <= d1:
-            return {"act_vs_kv_tokens": round(n0 + (n1 - n0) * (-d0) / (d1 - d0), 1)}
+            return {"act_vs_kv_tokens": round(n0 + (n1 - n0) * (-d0) / (d1 - d0), 1),
+                    "keep": "rp 0.5 (act) vs rkv 0.3 (kv)"}
     return {"act_vs_kv_tokens": None, "diff_ms": diff}
 
 
@@ -519,6 +581,58 @@ def run_kernel_only(args, local):
             "note": "includes the combine kernel" if args.only_kernel == "attention" else ""}
 
 
+SITES = {"dense": ["qkv", "attn", "o", "gate_up", "down"],
+         "act": ["sel_qkv", "qkv", "attn", "sel_o", "o", "sel_gu", "gate_up", "sel_d", "down"],
+         "kv": ["qkv", "page_scores", "page_select", "attn", "o", "gate_up", "down"],
+         "both": ["sel_qkv", "qkv", "page_scores", "page_select", "attn", "sel_o", "o", "sel_gu", "gate_up",
+                  "sel_d", "down"]}
+
+
+def run_timeline(args, local):
+    """Per-site cost of one decode step, from the kernel timestamps CUPTI
+    records (torch.profiler): with programmatic dependent launch a kernel's
+    CTAs start before its predecessor ends, so each site is charged the time
+    from the previous kernel's end to its own end."""
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+    import activation_kv_sparsity_b200 as bc
+    from synth import LLAMA_8B, kv_chunks, make_weights
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = LLAMA_8B
+    mode, n = args.timeline, args.contexts[0]
+    w = make_weights(cfg, seed=0, device=dev)
+    model = bc.Model(cfg, w, n + args.warmup + 8)
+    for k, v in kv_chunks(cfg, n, seed=1, device=dev):
+        model.append(k, v)
+    logits = torch.empty(cfg["vocab"], device=dev)
+    for i in range(args.warmup):
+        model.step(1 + i, mode, logits, **MODE_KW[mode])
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        model.step(7, mode, logits, **MODE_KW[mode])
+        torch.cuda.synchronize()
+    ev = [e for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA
+          and "k_" in e.name.split("(")[0]]
+    ev.sort(key=lambda e: e.time_range.start)
+    order = SITES[mode]
+    L = cfg["n_layers"]
+    if len(ev) != L * len(order) + 1:
+        return {"error": f"expected {L * len(order) + 1} kernels, traced {len(ev)}"}
+    cost = {k: 0.0 for k in order}
+    prev = ev[0].time_range.start
+    for i, e in enumerate(ev[:-1]):
+        cost[order[i % len(order)]] += e.time_range.end - prev
+        prev = e.time_range.end
+    span = (ev[-1].time_range.end - ev[0].time_range.start) / 1000.0
+    out = {"mode": mode, "context": n, "step_ms": round(span, 4),
+           "us_per_layer": {k: round(v / L, 2) for k, v in cost.items()},
+           "lm_head_us": round((ev[-1].time_range.end - prev) / 1.0, 2),
+           "note": "CUPTI kernel timestamps; each site charged from the previous kernel's end to its own end"}
+    model.close()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -529,6 +643,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--modes", nargs="+", default=["dense", "act", "kv", "both"],
                     choices=["dense", "act", "kv", "both"])
+    ap.add_argument("--timeline", choices=("dense", "act", "kv", "both"),
+                    help="per-site cost of one step in this mode at the first --contexts value")
     ap.add_argument("--only-kernel", choices=("gemv_gateup", "gemv_gateup_dense", "attention"),
                     help="time one kernel alone on a small case (profiler captures)")
     args = ap.parse_args()
@@ -543,6 +659,9 @@ def main():
     rank, ws, local = dist_init(args.gpus)
     if args.only_kernel:
         print(json.dumps(run_kernel_only(args, local)))
+        return
+    if args.timeline:
+        print(json.dumps(run_timeline(args, local)))
         return
     res = run_ours(args, rank, ws, local)
     if rank == 0:
