@@ -498,6 +498,13 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
     // attention block: [select] -> q/k/v GEMV (RMSNorm folded in; rotary,
     // append and page bounds in the epilogue) -> [page scores + select] ->
     // split-K attention with fused combine
+    // gate/up with the SwiGLU epilogue (h = silu(gate) * up written by the
+    // GEMV) when its column tiles pair whole channels; otherwise the down
+    // projection forms h from gate and up while staging
+    int tw_gu = 0, s_gu_ = 0, c_gu_ = 0;
+    gemv_plan(k_gu, 2 * f, m->sms, &tw_gu, &s_gu_, &c_gu_);
+    const bool sw = f % (tw_gu / 2) == 0;
+    float* d_in_vec = sw ? hmid : gu;
     if (act) {
       SelectArgs sa;
       BC_CUDA(step_select(m, first ? SP_EMBED_NORM : SP_NORM, d, k_qkv, x, g_attn, emb, x, xn, s_qkv, &sa),
@@ -564,15 +571,17 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
       ++launches;
     }
     BC_CUDA(step_gemv(m, 2, wgu + (size_t)l * d * 2 * f, d, 2 * f, GP_NORM, x, g_mlp, nullptr, nullptr,
-                      act ? s_gu : nullptr, k_gu, EPI_STORE, gu, nullptr, nullptr, nullptr), "gemv gate/up");
+                      act ? s_gu : nullptr, k_gu, sw ? EPI_SWIGLU : EPI_STORE, d_in_vec, nullptr, nullptr,
+                      nullptr), "gemv gate/up");
     ++launches;
     if (act) {
-      BC_CUDA(step_select(m, SP_SWIGLU, f, k_d, gu, nullptr, nullptr, nullptr, hmid, s_d, nullptr),
+      BC_CUDA(step_select(m, sw ? SP_NONE : SP_SWIGLU, f, k_d, d_in_vec, nullptr, nullptr, nullptr,
+                          sw ? nullptr : hmid, s_d, nullptr),
               "select down");
       ++launches;
     }
-    BC_CUDA(step_gemv(m, 3, wd + (size_t)l * f * d, f, d, GP_SWIGLU, gu, nullptr, nullptr, nullptr,
-                      act ? s_d : nullptr, k_d, EPI_RESID, x, xo, nullptr, nullptr), "gemv down");
+    BC_CUDA(step_gemv(m, 3, wd + (size_t)l * f * d, f, d, sw ? GP_NONE : GP_SWIGLU, d_in_vec, nullptr, nullptr,
+                      nullptr, act ? s_d : nullptr, k_d, EPI_RESID, x, xo, nullptr, nullptr), "gemv down");
     ++launches;
   }
   LmHeadArgs lm{static_cast<const __nv_bfloat16*>(m->w.lm_head), c.vocab, d, x,

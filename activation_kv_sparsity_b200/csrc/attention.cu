@@ -179,31 +179,68 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn(AttnArgs a) {
       mma16816(o[b], pa, b0, b1);
     }
   };
-  auto page_at = [&](int i) { return plist ? plist[i] : i; };
-  auto prefetch = [&](int i) {
-    if (lane == 0 && i < i_end)
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
-                   :: "l"(head_base + (size_t)page_at(i) * PAGE_ELEMS), "r"(PAGE_ELEMS * 2) : "memory");
+  // The warp's page numbers: iteration jj handles list entry
+  // i_begin + warp + kAttnWarps * jj.  A listed slice is held in two
+  // 32-entry register windows (lane l holds entries base + l and
+  // base + 32 + l), read by shuffles, so no page load waits on an index
+  // load; the window moves on by 32 entries long before they are needed.
+  auto entry = [&](int jj) {
+    const int i = i_begin + warp + kAttnWarps * jj;
+    return i < i_end ? plist[i] : 0;
+  };
+  int win0 = 0, win1 = 0, base = 0;
+  if (plist) {
+    win0 = entry(lane);
+    win1 = entry(32 + lane);
+  }
+  auto page_of = [&](int jj) {
+    if (!plist) return i_begin + warp + kAttnWarps * jj;
+    const int rel = jj - base;                       // warp-uniform, 0 <= rel < 64
+    return __shfl_sync(0xffffffffu, rel < 32 ? win0 : win1, rel & 31);
+  };
+  auto advance = [&](int jj) {                       // before looking up jj + 2
+    if (plist && jj + 2 - base >= 64) {
+      base += 32;
+      win0 = win1;
+      win1 = entry(base + 32 + lane);
+    }
+  };
+  const int n_it = i_begin + warp < i_end ? (i_end - i_begin - warp + kAttnWarps - 1) / kAttnWarps : 0;
+  auto prefetch = [&](int jj) {
+    if (jj < n_it) {
+      const int page = page_of(jj);
+      if (lane == 0)
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                     :: "l"(head_base + (size_t)page * PAGE_ELEMS), "r"(PAGE_ELEMS * 2) : "memory");
+    }
   };
 
   // ping-pong over two register buffers: the next page is in flight while
-  // this one is processed, and pages two steps ahead are pulled into L2
+  // this one is processed, and the page two steps ahead is pulled into L2
   uint4 ka0[U4], ka1[U4], va0[U4], va1[U4];
   uint4 kb0[U4], kb1[U4], vb0[U4], vb1[U4];
-  int i = i_begin + warp;
-  if (i < i_end) load_page(page_at(i), ka0, ka1, va0, va1);
-  while (i < i_end) {
-    int j = i + kAttnWarps;
-    prefetch(j + kAttnWarps);
-    if (j < i_end) load_page(page_at(j), kb0, kb1, vb0, vb1);
-    process_page(page_at(i), ka0, ka1, va0, va1);
-    i = j;
-    if (i >= i_end) break;
-    j = i + kAttnWarps;
-    prefetch(j + kAttnWarps);
-    if (j < i_end) load_page(page_at(j), ka0, ka1, va0, va1);
-    process_page(page_at(i), kb0, kb1, vb0, vb1);
-    i = j;
+  int pa_cur = 0, pb_cur = 0;
+  if (n_it > 0) {
+    pa_cur = page_of(0);
+    load_page(pa_cur, ka0, ka1, va0, va1);
+  }
+  for (int jj = 0; jj < n_it;) {
+    advance(jj);
+    prefetch(jj + 2);
+    if (jj + 1 < n_it) {
+      pb_cur = page_of(jj + 1);
+      load_page(pb_cur, kb0, kb1, vb0, vb1);
+    }
+    process_page(pa_cur, ka0, ka1, va0, va1);
+    if (++jj >= n_it) break;
+    advance(jj);
+    prefetch(jj + 2);
+    if (jj + 1 < n_it) {
+      pa_cur = page_of(jj + 1);
+      load_page(pa_cur, ka0, ka1, va0, va1);
+    }
+    process_page(pb_cur, kb0, kb1, vb0, vb1);
+    ++jj;
   }
 
   // this warp's state for head row g (lanes of a quad share it)
@@ -288,18 +325,19 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn(AttnArgs a) {
   }
   __syncthreads();
   // each thread owns 4 consecutive outputs (a float4) and sums the splits in
-  // order, 8 split loads in flight at a time
+  // order, up to 32 split loads in flight at a time
+  constexpr int kFly = 32;
   for (int e4 = threadIdx.x; e4 < G * HD / 4; e4 += kAttnWarps * 32) {
     const int hh = (e4 * 4) / HD, d = (e4 * 4) % HD;
     const float4* po = reinterpret_cast<const float4*>(a.part_o + (size_t)(h * G + hh) * kMaxSplits * HD + d);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sp0 = 0; sp0 < a.splits; sp0 += 8) {
-      float4 v[8];
+    for (int sp0 = 0; sp0 < a.splits; sp0 += kFly) {
+      float4 v[kFly];
       #pragma unroll
-      for (int u = 0; u < 8; ++u)
+      for (int u = 0; u < kFly; ++u)
         v[u] = sp0 + u < a.splits ? __ldcg(po + (size_t)(sp0 + u) * (HD / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
       #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < kFly; ++u) {
         const float w = sp0 + u < a.splits ? s_w[hh][sp0 + u] : 0.f;
         acc.x += w * v[u].x;
         acc.y += w * v[u].y;

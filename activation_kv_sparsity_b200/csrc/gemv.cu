@@ -28,6 +28,12 @@
 // takes an atomic ticket; the last to arrive (no spinning) sums the clusters'
 // partials in order.  Both stages sum in a fixed order: deterministic.  The
 // CTA that holds the tile's complete sum applies the epilogue:
+//   STORE   y = r
+//   RESID   y += r (the residual stream), optionally copied
+//   QKV     rotary embedding of q and k, bf16 append of k and v to their
+//           page, refresh of that page's key bounds
+//   SWIGLU  the tile pairs TW/2 gate columns with the up columns of the same
+//           channels, and y = silu(gate) * up for those channels
 #include "common.cuh"
 #include "kernels.h"
 
@@ -111,6 +117,11 @@ __device__ void qkv_epilogue(const QkvEpilogue& e, int col0, float v, float* s_v
   }
 }
 
+// x0^2 + x1^2 + x2^2 + x3^2 in one fixed order.
+__device__ __forceinline__ float sumsq4(float x0, float x1, float x2, float x3) {
+  return fmaf(x3, x3, fmaf(x2, x2, fmaf(x1, x1, x0 * x0)));
+}
+
 __device__ __forceinline__ float prep_value(const GemvArgs& a, int c) {
   switch (a.prep) {
     case GP_NORM: return a.x[c] * bf16f(a.gain[c]);
@@ -149,20 +160,34 @@ __global__ void __launch_bounds__(kGemvThreads, 2) k_gemv(GemvArgs a) {
   int* s_idx = reinterpret_cast<int*>(smem);
   float* s_x = reinterpret_cast<float*>(smem + sizeof(int) * a.max_rows);
   const bool norm = a.prep == GP_NORM || a.prep == GP_EMBED_NORM;
-  const __nv_bfloat16* wcol = a.W + col0 + lcol * 8;
+  // SWIGLU epilogue: the tile pairs gate columns t*TW/2 .. +TW/2 (lanes of
+  // the first half of a row) with the up columns of the same channels
+  const bool paired = a.epi == EPI_SWIGLU;
+  const int hcol0 = t * (TW / 2);
+  const __nv_bfloat16* wcol =
+      a.W + (!paired ? col0 + lcol * 8
+                     : (lcol < LPR / 2 ? hcol0 + lcol * 8 : a.d_out / 2 + hcol0 + (lcol - LPR / 2) * 8));
   const size_t ld = (size_t)a.d_out;
   const int my0 = warp * RPI + lrow;              // this lane's first row in the run
 
+  uint4 w0[kRowsInFlight];
+  float ss = 0.f;
   // Weights do not depend on the previous kernel: in dense mode pull the
   // rows after the first batch into L2 and issue this lane's first batch of
   // rows before waiting for it, so the stream overlaps the previous kernel's
   // tail.
-  uint4 w0[kRowsInFlight];
   bool first_loaded = false;
   if (!a.idx) {
-    for (int r = ROWS_STEP * kRowsInFlight + tid; r < min(nr, kPrefetchRowsL2); r += kGemvThreads)
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
-                   :: "l"(a.W + (size_t)(r0 + r) * ld + col0), "r"(TW * 2) : "memory");
+    for (int r = ROWS_STEP * kRowsInFlight + tid; r < min(nr, kPrefetchRowsL2); r += kGemvThreads) {
+      const __nv_bfloat16* row = a.W + (size_t)(r0 + r) * ld;
+      if (!paired) {
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(row + col0), "r"(TW * 2) : "memory");
+      } else {
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(row + hcol0), "r"(TW) : "memory");
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                     :: "l"(row + a.d_out / 2 + hcol0), "r"(TW) : "memory");
+      }
+    }
     #pragma unroll
     for (int u = 0; u < kRowsInFlight; ++u) {
       const int rr = my0 + u * ROWS_STEP;
@@ -188,14 +213,23 @@ __global__ void __launch_bounds__(kGemvThreads, 2) k_gemv(GemvArgs a) {
   }
 
   // RMSNorm statistics over the whole input: independent loads, 4 in flight
-  float ss = 0.f;
   if (norm) {
     if (a.prep == GP_NORM) {
       const float4* x4 = reinterpret_cast<const float4*>(a.x);
       #pragma unroll 4
       for (int c = tid; c < a.d_in / 4; c += kGemvThreads) {
         const float4 v = x4[c];
-        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+        ss += sumsq4(v.x, v.y, v.z, v.w);
+      }
+    } else if (a.d_in % 4 == 0) {
+      const uint2* e4 = reinterpret_cast<const uint2*>(a.embed_row);
+      #pragma unroll 4
+      for (int c = tid; c < a.d_in / 4; c += kGemvThreads) {
+        const uint2 e = e4[c];
+        const float e0 = bf16_lo(e.x), e1 = bf16_hi(e.x), e2 = bf16_lo(e.y), e3 = bf16_hi(e.y);
+        ss += sumsq4(e0, e1, e2, e3);
+        if (blockIdx.x == 0 && blockIdx.y == 0)
+          reinterpret_cast<float4*>(a.x_init)[c] = make_float4(e0, e1, e2, e3);
       }
     } else {
       #pragma unroll 4
@@ -327,6 +361,14 @@ __global__ void __launch_bounds__(kGemvThreads, 2) k_gemv(GemvArgs a) {
   if (a.epi == EPI_QKV) {
     if (tid < TW) a.y[col] = r;
     qkv_epilogue<TW>(a.qkv, col0, r, s_v);
+  } else if (a.epi == EPI_SWIGLU) {
+    // h = silu(gate) * up for the tile's TW/2 channels
+    if (tid < TW) s_v[tid] = r;
+    __syncthreads();
+    if (tid < TW / 2) {
+      const float g = s_v[tid], u = s_v[tid + TW / 2];
+      a.y[hcol0 + tid] = g / (1.0f + expf(-g)) * u;
+    }
   } else if (tid < TW) {
     if (a.epi == EPI_STORE) {
       a.y[col] = r;

@@ -11,7 +11,7 @@ namespace bc {
 void set_error(const char* msg);
 
 // ------------------------------------------------------------------ GEMV
-enum GemvEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_QKV = 2 };
+enum GemvEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_QKV = 2, EPI_SWIGLU = 3 };
 // How the GEMV input v is formed from x while staging (see gemv.cu).
 enum GemvPrep { GP_NONE = 0, GP_NORM = 1, GP_EMBED_NORM = 2, GP_SWIGLU = 3 };
 
@@ -43,7 +43,7 @@ struct GemvArgs {
   float* partial;            // [d_out/TW][kGemvMaxContrib][TW] (C > 1 only)
   unsigned* counters;        // [d_out / TW], zero between launches
   int epi;
-  float* y;                  // STORE: y = r; RESID: y += r; QKV: y = r (raw)
+  float* y;                  // STORE: y = r; RESID: y += r; QKV: y = r (raw); SWIGLU: h [d_out/2]
   float* y_copy;             // RESID: optional copy of the updated y
   QkvEpilogue qkv;
 };

@@ -15,194 +15,20 @@
 //   the best-scored others (README, "What it does in one picture": sinks,
 //   part of the history and the recent entries).
 //
-// Exact top-k over 32-bit order keys: an interval search that splits the
-// candidates' key range into 256 bins per pass.  Only the first pass sweeps
-// every key; the keys of the boundary bin are gathered into shared memory and
-// the remaining passes (at most four) run on them.  A single block scan over
-// packed (above-cut, at-cut) counts in index order then places every kept
-// index: ties at the cut go to the lower indices, and the list comes out
-// ascending.
+// Exact top-k over 32-bit order keys (topk.cuh): an interval search that
+// splits the candidates' key range into 256 bins per pass, then a placement
+// pass in index order, so ties at the cut go to the lower indices and the
+// list comes out ascending.  The cluster version below combines the passes
+// of the CTAs' slices through distributed shared memory.
 #include "common.cuh"
 #include "kernels.h"
+#include "topk.cuh"
 
 #include <cooperative_groups.h>
 
 namespace cg = cooperative_groups;
 
 namespace bc {
-
-enum : uint8_t { ST_OUT = 0, ST_CAND = 1, ST_FORCED = 2 };
-
-constexpr int kCandCap = 2048;   // boundary-bin candidates kept in shared memory
-
-template <int NT>
-struct TopkSmem {
-  int hist[256];
-  int red[32];
-  uint32_t rmin[32], rmax[32];
-  uint32_t cand_key[kCandCap];
-  int cand_n;
-  uint32_t bin;
-  int above, cnt;
-};
-
-// One pass of the interval search over `m` keys: counts them into at most 256
-// equal power-of-two-wide bins of [base, base + span_m1] and finds the bin
-// where the count from the top reaches rem.  Narrows the interval to that bin, lowers rem by the keys
-// above it and returns the bin's count.  All NT threads call it.
-template <int NT, typename KeyAt>
-__device__ int interval_pass(int m, KeyAt key_at, uint32_t& base, uint32_t& span_m1, int& rem,
-                             TopkSmem<NT>& sm) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // power-of-two bin width: the smallest 2^sh with (span_m1 >> sh) < 256
-  const int sh = max(0, 24 - __clz(span_m1));
-  const uint32_t width = 1u << sh;
-  for (int i = tid; i < m; i += NT) {
-    uint32_t kk;
-    if (!key_at(i, kk)) continue;
-    if (kk >= base && kk - base <= span_m1) atomicAdd(&sm.hist[(kk - base) >> sh], 1);
-  }
-  __syncthreads();
-  if (warp == 0) {
-    int c[8], sum = 0;
-    #pragma unroll
-    for (int j = 0; j < 8; ++j) {                 // lane owns bins 255-8*lane .. 248-8*lane
-      c[j] = sm.hist[255 - 8 * lane - j];
-      sum += c[j];
-    }
-    int incl = sum;
-    #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int above = incl - sum;
-    #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (above < rem && above + c[j] >= rem) {
-        sm.bin = (uint32_t)(255 - 8 * lane - j);
-        sm.above = above;
-        sm.cnt = c[j];
-      }
-      above += c[j];
-    }
-  }
-  __syncthreads();
-  const uint32_t b_lo = sm.bin * width;
-  rem -= sm.above;
-  const int cnt = sm.cnt;
-  base += b_lo;
-  span_m1 = min(width - 1u, span_m1 - b_lo);
-  for (int j = tid; j < 256; j += NT) sm.hist[j] = 0;
-  __syncthreads();
-  return cnt;
-}
-
-// Writes the forced elements and the `need` best candidates (by key, higher
-// first; ties to the lower index) of [0, n) to out, ascending.  All NT
-// threads must call it, each with the min and max key of the candidates it
-// saw (lo/hi; the block combines them), and sm.hist zeroed.
-//
-// The search keeps an interval [base, base + span_m1] of key values that
-// holds the cut: candidates above it are kept, below it dropped.  A pass
-// splits the interval into 256 equal bins and keeps the bin where the count
-// from the top reaches `need`, so the interval shrinks 256-fold per pass
-// until one key value is left or the bin is kept whole.  Starting from the
-// candidates' [min, max] spreads keys over the bins however their exponents
-// cluster.  Only the first pass sweeps all n keys: the boundary bin's keys
-// are then gathered into shared memory and the later passes run on them.
-template <int NT, typename KeyF, typename StateF>
-__device__ void radix_topk(int n, int need, KeyF key, StateF state, int* out, TopkSmem<NT>& sm,
-                           uint32_t lo, uint32_t hi) {
-  static_assert(NT >= 256 && NT % 32 == 0 && NT <= 1024, "block shape");
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint32_t base = 0, span_m1 = 0xFFFFFFFFu;
-  int rem = need;
-  if (need > 0) {
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-      hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-    }
-    if (lane == 0) {
-      sm.rmin[warp] = lo;
-      sm.rmax[warp] = hi;
-    }
-    if (tid == 0) sm.cand_n = 0;
-    __syncthreads();
-    lo = 0xFFFFFFFFu;
-    hi = 0u;
-    #pragma unroll
-    for (int w = 0; w < NT / 32; ++w) {
-      lo = min(lo, sm.rmin[w]);
-      hi = max(hi, sm.rmax[w]);
-    }
-    base = lo;
-    span_m1 = hi - lo;
-    auto full = [&](int i, uint32_t& kk) {
-      if (state(i) != ST_CAND) return false;
-      kk = key(i);
-      return true;
-    };
-    int cnt = span_m1 > 0 ? interval_pass<NT>(n, full, base, span_m1, rem, sm) : 0;
-    if (span_m1 > 0 && cnt != rem) {
-      if (cnt <= kCandCap) {
-        // gather the boundary bin's keys, then narrow on them alone
-        for (int i = tid; i < n; i += NT) {
-          if (state(i) != ST_CAND) continue;
-          const uint32_t kk = key(i);
-          if (kk >= base && kk - base <= span_m1) sm.cand_key[atomicAdd(&sm.cand_n, 1)] = kk;
-        }
-        __syncthreads();
-        const int m = sm.cand_n;
-        auto small = [&](int i, uint32_t& kk) {
-          kk = sm.cand_key[i];
-          return true;
-        };
-        #pragma unroll 1
-        for (int pass = 0; pass < 4 && span_m1 > 0; ++pass)
-          if (interval_pass<NT>(m, small, base, span_m1, rem, sm) == rem) break;
-      } else {
-        #pragma unroll 1
-        for (int pass = 0; pass < 4 && span_m1 > 0; ++pass)
-          if (interval_pass<NT>(n, full, base, span_m1, rem, sm) == rem) break;
-      }
-    }
-  }
-  // keep: key above the interval, or inside it among the first `rem` by index
-  const uint32_t top = base + span_m1;            // inclusive upper end
-  const int per = (n + NT - 1) / NT;
-  const int b0 = min(n, tid * per), b1 = min(n, b0 + per);
-  int gt = 0, eq = 0;
-  for (int i = b0; i < b1; ++i) {
-    const uint8_t st = state(i);
-    if (st == ST_FORCED) {
-      ++gt;
-    } else if (st == ST_CAND && need > 0) {
-      const uint32_t kk = key(i);
-      gt += kk > top;
-      eq += kk >= base && kk <= top;
-    }
-  }
-  int total;
-  const int excl = block_excl_scan<NT>((gt << 16) | eq, sm.red, &total);
-  int er = excl & 0xFFFF;
-  int pos = (excl >> 16) + min(er, rem);
-  for (int i = b0; i < b1; ++i) {
-    const uint8_t st = state(i);
-    bool keep = st == ST_FORCED;
-    if (st == ST_CAND && need > 0) {
-      const uint32_t kk = key(i);
-      if (kk > top) {
-        keep = true;
-      } else if (kk >= base) {
-        keep = er < rem;
-        ++er;
-      }
-    }
-    if (keep) out[pos++] = i;
-  }
-}
 
 // ------------------------------------------------------------------ activation select
 // Above 8192 elements a cluster of kSelCluster CTAs (one per SM) ranks one vector: CTA r owns the
@@ -502,6 +328,34 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl) {
 // are in flight while the current round is scored.
 constexpr int kPageThreads = 256;
 
+// The page bound of one page for the group's query heads: the max over
+// heads of sum_c max(q_c * kmin_c, q_c * kmax_c).  The LPP lanes of a page
+// each hold 8 channels (mn/mx: their 8 bf16 bounds); every lane of the group
+// returns the page's score.
+template <int LPP, int GMAX>
+__device__ __forceinline__ float page_bound_score(const float (&qv)[GMAX][8], int G, const uint4& mn,
+                                                  const uint4& mx) {
+  const uint32_t mnw[4] = {mn.x, mn.y, mn.z, mn.w};
+  const uint32_t mxw[4] = {mx.x, mx.y, mx.z, mx.w};
+  float best = -INFINITY;
+  #pragma unroll
+  for (int g = 0; g < GMAX; ++g) {
+    if (g >= G) break;
+    float s = 0.f;
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float lo0 = bf16_lo(mnw[j]), lo1 = bf16_hi(mnw[j]);
+      const float hi0 = bf16_lo(mxw[j]), hi1 = bf16_hi(mxw[j]);
+      s += fmaxf(qv[g][2 * j] * lo0, qv[g][2 * j] * hi0);
+      s += fmaxf(qv[g][2 * j + 1] * lo1, qv[g][2 * j + 1] * hi1);
+    }
+    #pragma unroll
+    for (int o = LPP / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o, LPP);
+    best = fmaxf(best, s);
+  }
+  return best;
+}
+
 template <int HD>
 __host__ __device__ constexpr int pages_per_round() {
   return (kPageThreads / 32) * (32 / (HD / 8)) * 4;
@@ -551,24 +405,7 @@ __global__ void __launch_bounds__(kPageThreads, GMAX <= 4 ? 2 : 1) k_pages(PageA
     #pragma unroll
     for (int it = 0; it < STEPS; ++it) {
       const int p = page_of(round, it);
-      const uint32_t mnw[4] = {mn[it].x, mn[it].y, mn[it].z, mn[it].w};
-      const uint32_t mxw[4] = {mx[it].x, mx[it].y, mx[it].z, mx[it].w};
-      float best = -INFINITY;
-      #pragma unroll
-      for (int g = 0; g < GMAX; ++g) {
-        if (g >= a.G) break;
-        float s = 0.f;
-        #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float lo0 = bf16_lo(mnw[j]), lo1 = bf16_hi(mnw[j]);
-          const float hi0 = bf16_lo(mxw[j]), hi1 = bf16_hi(mxw[j]);
-          s += fmaxf(qv[g][2 * j] * lo0, qv[g][2 * j] * hi0);
-          s += fmaxf(qv[g][2 * j + 1] * lo1, qv[g][2 * j + 1] * hi1);
-        }
-        #pragma unroll
-        for (int o = LPP / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o, LPP);
-        best = fmaxf(best, s);
-      }
+      const float best = page_bound_score<LPP, GMAX>(qv, a.G, mn[it], mx[it]);
       if (p < a.P && cl == 0) scores[p] = best;
     }
   };

@@ -581,11 +581,23 @@ def run_kernel_only(args, local):
             "note": "includes the combine kernel" if args.only_kernel == "attention" else ""}
 
 
-SITES = {"dense": ["qkv", "attn", "o", "gate_up", "down"],
-         "act": ["sel_qkv", "qkv", "attn", "sel_o", "o", "sel_gu", "gate_up", "sel_d", "down"],
-         "kv": ["qkv", "page_scores", "page_select", "attn", "o", "gate_up", "down"],
-         "both": ["sel_qkv", "qkv", "page_scores", "page_select", "attn", "sel_o", "o", "sel_gu", "gate_up",
-                  "sel_d", "down"]}
+GEMV_SITES = ["qkv", "o", "gate_up", "down"]
+
+
+def site_of(kernel: str, gemvs_seen: int) -> str:
+    """Step site of a traced kernel: GEMVs come in projection order within a
+    layer, a selection kernel belongs to the GEMV after it."""
+    if "k_gemv" in kernel:
+        return GEMV_SITES[gemvs_seen % 4]
+    if "k_page_select" in kernel:
+        return "page_select"
+    if "k_pages" in kernel:
+        return "page_scores"
+    if "k_select" in kernel:
+        return "sel_" + GEMV_SITES[gemvs_seen % 4]
+    if "k_attn" in kernel:
+        return "attn"
+    return kernel
 
 
 def run_timeline(args, local):
@@ -615,17 +627,20 @@ def run_timeline(args, local):
     ev = [e for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA
           and "k_" in e.name.split("(")[0]]
     ev.sort(key=lambda e: e.time_range.start)
-    order = SITES[mode]
     L = cfg["n_layers"]
-    if len(ev) != L * len(order) + 1:
-        return {"error": f"expected {L * len(order) + 1} kernels, traced {len(ev)}"}
-    cost = {k: 0.0 for k in order}
+    if not ev or "k_lmhead" not in ev[-1].name:
+        return {"error": f"the step's last kernel is not the LM head ({len(ev)} traced)"}
+    cost = {}
+    gemvs = 0
     prev = ev[0].time_range.start
-    for i, e in enumerate(ev[:-1]):
-        cost[order[i % len(order)]] += e.time_range.end - prev
+    for e in ev[:-1]:
+        name = e.name.split("(")[0]
+        site = site_of(name, gemvs)
+        gemvs += "k_gemv" in name
+        cost[site] = cost.get(site, 0.0) + e.time_range.end - prev
         prev = e.time_range.end
     span = (ev[-1].time_range.end - ev[0].time_range.start) / 1000.0
-    out = {"mode": mode, "context": n, "step_ms": round(span, 4),
+    out = {"mode": mode, "context": n, "step_ms": round(span, 4), "kernels": len(ev),
            "us_per_layer": {k: round(v / L, 2) for k, v in cost.items()},
            "lm_head_us": round((ev[-1].time_range.end - prev) / 1.0, 2),
            "note": "CUPTI kernel timestamps; each site charged from the previous kernel's end to its own end"}
