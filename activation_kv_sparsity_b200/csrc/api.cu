@@ -187,6 +187,7 @@ struct NodeRec {
 // A captured decode step for one (mode, rp, rkv, sinks, recent).
 struct StepGraph {
   bc_mode mode;
+  int psel;              // page-select variant of the captured page counts (kv modes)
   float rp, rkv;
   int sinks, recent;
   cudaGraph_t graph;
@@ -599,6 +600,7 @@ static bc_status capture_step(bc_model* m, int token, bc_mode mode, float rp, fl
   if (!m->cap_stream) BC_CUDA(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking), "capture stream");
   StepGraph* g = new StepGraph();
   g->mode = mode;
+  g->psel = 0;
   g->rp = rp;
   g->rkv = rkv;
   g->sinks = sinks;
@@ -678,8 +680,12 @@ static bc_status run_step(bc_model* m, int token, bc_mode mode, float rp, float 
   const StepShape sh = step_shape(m, mode, rp, rkv, sinks, recent);
   if (m->use_graphs) {
     StepGraph* g = nullptr;
+    const bool kvs = mode == BC_KV || mode == BC_BOTH;
+    const int psel = kvs ? page_select_variant(sh.P) : 0;
     for (StepGraph* c : m->graphs)
-      if (c->mode == mode && c->rp == rp && c->rkv == rkv && c->sinks == sinks && c->recent == recent) g = c;
+      if (c->mode == mode && c->psel == psel && c->rp == rp && c->rkv == rkv && c->sinks == sinks &&
+          c->recent == recent)
+        g = c;
     if (g) {
       cudaError_t e = launch_step_graph(m, g, token, sh, logits);
       if (e == cudaSuccess) {
@@ -693,6 +699,7 @@ static bc_status run_step(bc_model* m, int token, bc_mode mode, float rp, float 
     } else if (m->launches > 0) {
       // the kernels' attributes are set up by an earlier direct step: capture now
       if (capture_step(m, token, mode, rp, rkv, sinks, recent, logits, &g) == BC_OK) {
+        g->psel = psel;
         m->graphs.push_back(g);
         if (launch_step_graph(m, g, token, sh, logits) == cudaSuccess) {
           commit_step(m, mode, sh, g->launches);

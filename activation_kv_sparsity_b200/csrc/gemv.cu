@@ -48,7 +48,6 @@ namespace bc {
 constexpr int kGemvWarps = 8;
 constexpr int kGemvThreads = kGemvWarps * 32;
 constexpr int kRowsInFlight = 16;
-constexpr int kPrefetchRowsL2 = 512;   // dense rows per CTA pulled into L2 before the dependency wait
 
 __device__ __forceinline__ void fma8(float* acc, float xv, const uint4& w) {
   acc[0] = fmaf(xv, bf16_lo(w.x), acc[0]);
@@ -172,22 +171,12 @@ __global__ void __launch_bounds__(kGemvThreads, 2) k_gemv(GemvArgs a) {
 
   uint4 w0[kRowsInFlight];
   float ss = 0.f;
-  // Weights do not depend on the previous kernel: in dense mode pull the
-  // rows after the first batch into L2 and issue this lane's first batch of
-  // rows before waiting for it, so the stream overlaps the previous kernel's
-  // tail.
+  // Weights do not depend on the previous kernel: in dense mode issue this
+  // lane's first batch of rows before waiting for it, so the stream overlaps
+  // the previous kernel's tail.  (Pulling further rows into L2 as well was
+  // measured to cost more than it saved.)
   bool first_loaded = false;
   if (!a.idx) {
-    for (int r = ROWS_STEP * kRowsInFlight + tid; r < min(nr, kPrefetchRowsL2); r += kGemvThreads) {
-      const __nv_bfloat16* row = a.W + (size_t)(r0 + r) * ld;
-      if (!paired) {
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(row + col0), "r"(TW * 2) : "memory");
-      } else {
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(row + hcol0), "r"(TW) : "memory");
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
-                     :: "l"(row + a.d_out / 2 + hcol0), "r"(TW) : "memory");
-      }
-    }
     #pragma unroll
     for (int u = 0; u < kRowsInFlight; ++u) {
       const int rr = my0 + u * ROWS_STEP;

@@ -70,7 +70,8 @@ struct SelectArgs {
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl);
 
 // ------------------------------------------------------------------ KV pages
-// Page scores (grid-wide), then the page select (one cluster per kv head).
+// Page scores (grid-wide), then the page select (one CTA, or above 8192
+// pages one cluster, per kv head).
 struct PageArgs {
   const float* q;                 // rotated queries [Hkv*G][hd]
   const __nv_bfloat16* meta;      // layer key bounds [Hkv][Pmax][2][hd]
@@ -82,6 +83,10 @@ struct PageArgs {
 };
 cudaError_t launch_page_scores(const PageArgs& a, cudaStream_t st, bool pdl);
 cudaError_t launch_page_select(const PageArgs& a, cudaStream_t st, bool pdl);
+// Which page-select kernel P pages take: keys per thread of the one-CTA
+// kernel (2, 4 or 8), or 0 for the cluster.  A captured step serves only
+// page counts of its own variant.
+int page_select_variant(int P);
 // Launch shape of the page scorer for P pages (graph node updates).
 int page_rounds(int P, int hd, int Hkv, int sms);
 dim3 pages_grid(const PageArgs& a);

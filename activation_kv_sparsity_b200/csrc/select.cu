@@ -11,15 +11,19 @@
 //   the page key bound of Quest, listed among the paper's closest ancestors
 //   on its mlsanity page): s_p = max over the group's query heads of
 //   sum_c max(q_c*kmin_pc, q_c*kmax_pc).
-// * Page select, one cluster per kv head: forced sinks and recent pages plus
-//   the best-scored others (README, "What it does in one picture": sinks,
-//   part of the history and the recent entries).
+// * Page select, per kv head (one CTA up to 8192 pages, else a cluster):
+//   forced sinks and recent pages plus the best-scored others (README, "What
+//   it does in one picture": sinks, part of the history and the recent
+//   entries).
 //
-// Exact top-k over 32-bit order keys (topk.cuh): an interval search that
-// splits the candidates' key range into 256 bins per pass, then a placement
-// pass in index order, so ties at the cut go to the lower indices and the
-// list comes out ascending.  The cluster version below combines the passes
-// of the CTAs' slices through distributed shared memory.
+// Exact top-k over 32-bit order keys: an interval search that splits the
+// candidates' key range into 256 bins per pass, then a placement pass in
+// index order, so ties at the cut go to the lower indices and the list comes
+// out ascending.  One CTA ranks a vector of up to 8192 elements, or a kv
+// head's scores of up to 8192 pages, with its keys in registers (topk.cuh);
+// the cluster version below spreads a longer vector, or more pages, over the
+// CTAs of a cluster and combines the passes of their slices through
+// distributed shared memory.
 #include "common.cuh"
 #include "kernels.h"
 #include "topk.cuh"
@@ -60,25 +64,11 @@ template <typename StateF>
 __device__ void cluster_topk(const uint32_t* s_key, int s0, int ns, int need, StateF state, uint32_t lo,
                              uint32_t hi, int* out, SelClusterSmem& sm, cg::cluster_group& cl) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-  }
-  if (lane == 0) {
-    sm.rmin[warp] = lo;
-    sm.rmax[warp] = hi;
-  }
   for (int b = tid; b < 2 * 256; b += kSelClThreads) (&sm.hist[0][0])[b] = 0;
-  __syncthreads();
+  block_minmax<kSelClThreads>(lo, hi, sm.rmin, sm.rmax);
   if (tid == 0) {
-    uint32_t l2 = 0xFFFFFFFFu, h2 = 0u;
-    for (int w = 0; w < kSelClThreads / 32; ++w) {
-      l2 = min(l2, sm.rmin[w]);
-      h2 = max(h2, sm.rmax[w]);
-    }
-    sm.lo = l2;
-    sm.hi = h2;
+    sm.lo = lo;
+    sm.hi = hi;
   }
   cl.sync();
   lo = 0xFFFFFFFFu;
@@ -241,56 +231,53 @@ __global__ void __launch_bounds__(kSelClThreads, 1) k_select(SelectArgs a) {
   cluster_topk(s_key, s0, ns, a.k, [](int) { return (uint8_t)ST_CAND; }, lo, hi, a.idx, sm, cl);
 }
 
-// Vectors up to kSelOneCta elements: one CTA ranks the whole vector (a
-// cluster's barriers cost more than they save at this size).
+// Vectors up to kSelOneCta elements: one CTA ranks the whole vector with its
+// keys in registers (a cluster's barriers cost more than they save at this
+// size).  Warp w loads the elements (w*KPT + c)*32 + lane, c < KPT: rows of
+// 32 consecutive elements, all KPT rows in flight together.
 constexpr int kSelOneCta = 8192;
 constexpr int kSelThreads1 = 1024;
 
+template <int KPT>
 __global__ void __launch_bounds__(kSelThreads1, 1) k_select_cta(SelectArgs a) {
-  __shared__ uint32_t s_key[kSelOneCta];
-  __shared__ TopkSmem<kSelThreads1> sm;
+  __shared__ RegTopkSmem<kSelThreads1> sm;
   const int tid = threadIdx.x, n = a.n;
+  const int ibase = (tid >> 5) * KPT * 32 + (tid & 31);
   pdl_wait();
   pdl_trigger();
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  for (int j = tid; j < 256; j += kSelThreads1) sm.hist[j] = 0;
-  for (int i0 = 0; i0 < n; i0 += 8 * kSelThreads1) {
-    float a0[8], a1[8];
-    #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kSelThreads1 + tid;
-      a0[u] = 0.f;
-      a1[u] = 0.f;
-      if (i < n) {
-        switch (a.prep) {
-          case SP_NORM: a0[u] = a.x[i]; a1[u] = bf16f(a.gain[i]); break;
-          case SP_EMBED_NORM: a0[u] = bf16f(a.embed_row[i]); a1[u] = bf16f(a.gain[i]); break;
-          case SP_SWIGLU: a0[u] = a.x[i]; a1[u] = a.x[n + i]; break;
-          default: a0[u] = a.x[i];
-        }
-      }
-    }
-    #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kSelThreads1 + tid;
-      if (i >= n) break;
-      float v;
+  float a0[KPT], a1[KPT];
+  #pragma unroll
+  for (int c = 0; c < KPT; ++c) {
+    const int i = ibase + 32 * c;
+    a0[c] = 0.f;
+    a1[c] = 0.f;
+    if (i < n) {
       switch (a.prep) {
-        case SP_NORM: v = a0[u] * a1[u]; break;
-        case SP_EMBED_NORM: a.x_init[i] = a0[u]; v = a0[u] * a1[u]; break;
-        case SP_SWIGLU: v = a0[u] / (1.0f + expf(-a0[u])) * a1[u]; break;
-        default: v = a0[u];
+        case SP_NORM: a0[c] = a.x[i]; a1[c] = bf16f(a.gain[i]); break;
+        case SP_EMBED_NORM: a0[c] = bf16f(a.embed_row[i]); a1[c] = bf16f(a.gain[i]); break;
+        case SP_SWIGLU: a0[c] = a.x[i]; a1[c] = a.x[n + i]; break;
+        default: a0[c] = a.x[i];
       }
-      if (a.vout) a.vout[i] = v;
-      const uint32_t kk = __float_as_uint(fabsf(v));
-      s_key[i] = kk;
-      lo = min(lo, kk);
-      hi = max(hi, kk);
     }
   }
-  __syncthreads();
-  radix_topk<kSelThreads1>(
-      n, a.k, [&](int i) { return s_key[i]; }, [](int) { return (uint8_t)ST_CAND; }, a.idx, sm, lo, hi);
+  uint32_t kr[KPT];
+  #pragma unroll
+  for (int c = 0; c < KPT; ++c) {
+    const int i = ibase + 32 * c;
+    float v;
+    switch (a.prep) {
+      case SP_NORM: v = a0[c] * a1[c]; break;
+      case SP_EMBED_NORM: v = a0[c] * a1[c]; break;
+      case SP_SWIGLU: v = a0[c] / (1.0f + expf(-a0[c])) * a1[c]; break;
+      default: v = a0[c];
+    }
+    if (i < n) {
+      if (a.prep == SP_EMBED_NORM) a.x_init[i] = a0[c];
+      if (a.vout) a.vout[i] = v;
+    }
+    kr[c] = __float_as_uint(fabsf(v));
+  }
+  reg_topk<kSelThreads1, KPT>(kr, n, a.k, [](int) { return (uint8_t)ST_CAND; }, a.idx, sm);
 }
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl) {
@@ -304,7 +291,8 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl) {
     attr1[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr1;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, k_select_cta, a);
+    if (a.n <= kSelThreads1 * 4) return cudaLaunchKernelEx(&cfg, k_select_cta<4>, a);
+    return cudaLaunchKernelEx(&cfg, k_select_cta<8>, a);
   }
   cfg.gridDim = dim3(kSelCluster);
   cfg.blockDim = dim3(kSelClThreads);
@@ -329,31 +317,60 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl) {
 constexpr int kPageThreads = 256;
 
 // The page bound of one page for the group's query heads: the max over
-// heads of sum_c max(q_c * kmin_c, q_c * kmax_c).  The LPP lanes of a page
-// each hold 8 channels (mn/mx: their 8 bf16 bounds); every lane of the group
-// returns the page's score.
+// heads of sum_c max(q_c * kmin_c, q_c * kmax_c) = sum_c q_c * (q_c >= 0 ?
+// kmax_c : kmin_c).  The LPP lanes of a page each hold 8 channels (mn/mx:
+// their 8 bf16 bounds) and sum them for every head; a transpose-reduce then
+// halves the heads a lane carries at each of the first log2(GMAX) butterfly
+// steps (it keeps one half and sends the other), so all GMAX sums complete
+// in about GMAX + log2(LPP / GMAX) shuffles instead of GMAX * log2(LPP),
+// and a last butterfly takes the max over the heads.  Every lane of the page
+// returns the page's score.  Heads g >= G count as -inf.
 template <int LPP, int GMAX>
 __device__ __forceinline__ float page_bound_score(const float (&qv)[GMAX][8], int G, const uint4& mn,
                                                   const uint4& mx) {
+  static_assert(GMAX <= LPP, "one head per lane after the transpose");
   const uint32_t mnw[4] = {mn.x, mn.y, mn.z, mn.w};
   const uint32_t mxw[4] = {mx.x, mx.y, mx.z, mx.w};
-  float best = -INFINITY;
+  float lo[8], hi[8];
+  #pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    lo[2 * j] = bf16_lo(mnw[j]);
+    lo[2 * j + 1] = bf16_hi(mnw[j]);
+    hi[2 * j] = bf16_lo(mxw[j]);
+    hi[2 * j + 1] = bf16_hi(mxw[j]);
+  }
+  float v[GMAX];
   #pragma unroll
   for (int g = 0; g < GMAX; ++g) {
-    if (g >= G) break;
-    float s = 0.f;
+    float t = 0.f;
     #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float lo0 = bf16_lo(mnw[j]), lo1 = bf16_hi(mnw[j]);
-      const float hi0 = bf16_lo(mxw[j]), hi1 = bf16_hi(mxw[j]);
-      s += fmaxf(qv[g][2 * j] * lo0, qv[g][2 * j] * hi0);
-      s += fmaxf(qv[g][2 * j + 1] * lo1, qv[g][2 * j + 1] * hi1);
-    }
-    #pragma unroll
-    for (int o = LPP / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o, LPP);
-    best = fmaxf(best, s);
+    for (int c = 0; c < 8; ++c) t = fmaf(qv[g][c], qv[g][c] >= 0.f ? hi[c] : lo[c], t);
+    v[g] = t;
   }
-  return best;
+  const int lane = threadIdx.x & 31;
+  // transpose-reduce: at offset o = LPP/2, LPP/4, ... a lane keeps the lower
+  // or upper half of its heads (by the lane bit o) and adds its partner's
+  // copy of that half
+  int head = 0;
+  #pragma unroll
+  for (int n = GMAX, o = LPP / 2; n > 1; n >>= 1, o >>= 1) {
+    const bool upper = (lane & o) != 0;
+    #pragma unroll
+    for (int j = 0; j < n / 2; ++j) {
+      const float send = upper ? v[j] : v[j + n / 2];
+      const float keep = upper ? v[j + n / 2] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+    head = 2 * head + (upper ? 1 : 0);
+  }
+  float s = v[0];
+  #pragma unroll
+  for (int o = LPP / (2 * GMAX); o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  // head now names the sum this lane holds; max over the heads
+  s = head < G ? s : -INFINITY;
+  #pragma unroll
+  for (int o = LPP / GMAX; o < LPP; o <<= 1) s = fmaxf(s, __shfl_xor_sync(0xffffffffu, s, o));
+  return s;
 }
 
 template <int HD>
@@ -420,8 +437,9 @@ __global__ void __launch_bounds__(kPageThreads, GMAX <= 4 ? 2 : 1) k_pages(PageA
   }
 }
 
-// Page select: one cluster per kv head; CTA r ranks the r-th slice of the
-// head's page scores.  Forced pages (sinks, recent) are kept and not ranked.
+// Page select above 8192 pages: one cluster per kv head; CTA r ranks the
+// r-th slice of the head's page scores.  Forced pages (sinks, recent) are
+// kept and not ranked.  (One CTA with 16 keys a thread measured slower.)
 __global__ void __launch_bounds__(kSelClThreads, 1) k_page_select(PageArgs a) {
   __shared__ uint32_t s_key[kSelSlice];
   __shared__ SelClusterSmem sm;
@@ -453,6 +471,30 @@ __global__ void __launch_bounds__(kSelClThreads, 1) k_page_select(PageArgs a) {
       a.pages + (size_t)h * a.Pmax, sm, cl);
 }
 
+// Page select up to 8192 pages, one CTA per kv head: the head's P scores as
+// register keys (KPT per thread, P <= 1024*KPT), forced pages kept.
+template <int KPT>
+__global__ void __launch_bounds__(kSelThreads1, 1) k_page_select_cta(PageArgs a) {
+  __shared__ RegTopkSmem<kSelThreads1> sm;
+  const int h = blockIdx.x, tid = threadIdx.x, P = a.P;
+  const int ibase = (tid >> 5) * KPT * 32 + (tid & 31);
+  pdl_wait();
+  pdl_trigger();
+  const float* scores = a.scores + (size_t)h * a.Pmax;
+  float v[KPT];
+  #pragma unroll
+  for (int c = 0; c < KPT; ++c) v[c] = ibase + 32 * c < P ? scores[ibase + 32 * c] : 0.f;
+  uint32_t kr[KPT];
+  #pragma unroll
+  for (int c = 0; c < KPT; ++c) kr[c] = float_order_key(v[c]);
+  const int sink_end = min(a.sinks, P), rec_begin = max(P - a.recent, 0);
+  const int n_forced = sink_end + (P - max(rec_begin, sink_end));
+  reg_topk<kSelThreads1, KPT>(
+      kr, P, a.K - n_forced,
+      [&](int i) { return (uint8_t)((i < sink_end || i >= rec_begin) ? ST_FORCED : ST_CAND); },
+      a.pages + (size_t)h * a.Pmax, sm);
+}
+
 int page_rounds(int P, int hd, int Hkv, int sms) {
   const int ppr = hd == 128 ? pages_per_round<128>() : pages_per_round<64>();
   const int units = Hkv * ((P + ppr - 1) / ppr);          // rounds of work in all
@@ -481,19 +523,36 @@ cudaError_t launch_page_scores(const PageArgs& a, cudaStream_t st, bool pdl) {
   return cudaErrorInvalidValue;
 }
 
+int page_select_variant(int P) {
+  if (P <= kSelThreads1 * 2) return 2;
+  if (P <= kSelThreads1 * 4) return 4;
+  if (P <= kSelThreads1 * 8) return 8;
+  return 0;
+}
+
 cudaError_t launch_page_select(const PageArgs& a, cudaStream_t st, bool pdl) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kSelCluster, a.Hkv);
-  cfg.blockDim = dim3(kSelClThreads);
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kSelCluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  const int variant = page_select_variant(a.P);
+  if (variant) {
+    cfg.gridDim = dim3(a.Hkv);
+    cfg.blockDim = dim3(kSelThreads1);
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (variant == 2) return cudaLaunchKernelEx(&cfg, k_page_select_cta<2>, a);
+    if (variant == 4) return cudaLaunchKernelEx(&cfg, k_page_select_cta<4>, a);
+    return cudaLaunchKernelEx(&cfg, k_page_select_cta<8>, a);
+  }
+  cfg.gridDim = dim3(kSelCluster, a.Hkv);
+  cfg.blockDim = dim3(kSelClThreads);
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = kSelCluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = pdl ? attr : attr + 1;
   cfg.numAttrs = pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, k_page_select, a);
 }

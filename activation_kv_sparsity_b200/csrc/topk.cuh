@@ -1,16 +1,23 @@
-// Exact top-k inside one CTA, shared by the selection kernels and the GEMV
-// that ranks its own input.
+// Exact top-k of one vector inside one CTA, keys held in registers.
 //
-// Keys are 32-bit order keys.  The cut is found by an interval search that
-// splits the candidates' key range into 256 bins per pass.  Only the first
-// pass sweeps every key; the keys of the boundary bin are gathered into
-// shared memory and the remaining passes (at most four) run on them.
-// Placement then walks the vector in index order, a warp per contiguous
-// segment and 32 elements per ballot: an element is kept when it is forced,
-// its key lies above the cut interval, or it is among the first `rem` keys
-// inside the interval by index.  Its slot in the ascending output is the
-// number of kept elements before it, so ties at the cut go to the lower
-// indices and the list comes out ascending.
+// Keys are 32-bit order keys.  Warp w owns the KPT*32 consecutive elements
+// from w*KPT*32; lane l holds in kr[c] the key of element (w*KPT + c)*32 + l,
+// so every load, ballot and store below is one coalesced row of 32 elements.
+//
+// The cut is found by an interval search: a pass counts the keys inside the
+// current interval [base, base + span] into 256 equal power-of-two-wide
+// bins and keeps the bin where the count from the top reaches the number
+// still needed; the interval shrinks 256-fold per pass, starting from the
+// keys' [min, max], until one key value is left or the boundary bin is kept
+// whole.  A pass costs one barrier: every warp reads the finished histogram
+// and finds the bin itself, and three histograms rotate so that the one
+// being cleared is never the one being counted into or read.
+//
+// Placement walks the elements in index order: an element is kept when its
+// key lies above the interval, or it is among the first `rem` keys inside it
+// by index; its slot in the ascending output is the number of kept elements
+// before it (ballots within a warp, a masked sum across warps), so ties at
+// the cut go to the lower indices and the list comes out ascending.
 #pragma once
 
 #include "common.cuh"
@@ -19,204 +26,154 @@ namespace bc {
 
 enum : uint8_t { ST_OUT = 0, ST_CAND = 1, ST_FORCED = 2 };
 
-constexpr int kCandCap = 2048;   // boundary-bin candidates kept in shared memory
-
+// Block-wide min of lo and max of hi, returned to every thread (one barrier).
 template <int NT>
-struct TopkSmem {
-  int hist[256];
-  int red[32];
-  int wtot[2][32];
-  uint32_t rmin[32], rmax[32];
-  uint32_t cand_key[kCandCap];
-  int cand_n;
-  uint32_t bin;
-  int above, cnt;
-};
-
-// One pass of the interval search over `m` keys: counts them into at most 256
-// equal power-of-two-wide bins of [base, base + span_m1] and finds the bin
-// where the count from the top reaches rem.  Narrows the interval to that
-// bin, lowers rem by the keys above it and returns the bin's count.  All NT
-// threads call it.
-template <int NT, typename KeyAt>
-__device__ int interval_pass(int m, KeyAt key_at, uint32_t& base, uint32_t& span_m1, int& rem,
-                             TopkSmem<NT>& sm) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // power-of-two bin width: the smallest 2^sh with (span_m1 >> sh) < 256
-  const int sh = max(0, 24 - __clz(span_m1));
-  const uint32_t width = 1u << sh;
-  for (int i = tid; i < m; i += NT) {
-    uint32_t kk;
-    if (!key_at(i, kk)) continue;
-    if (kk >= base && kk - base <= span_m1) atomicAdd(&sm.hist[(kk - base) >> sh], 1);
-  }
-  __syncthreads();
-  if (warp == 0) {
-    int c[8], sum = 0;
-    #pragma unroll
-    for (int j = 0; j < 8; ++j) {                 // lane owns bins 255-8*lane .. 248-8*lane
-      c[j] = sm.hist[255 - 8 * lane - j];
-      sum += c[j];
-    }
-    int incl = sum;
-    #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int above = incl - sum;
-    #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (above < rem && above + c[j] >= rem) {
-        sm.bin = (uint32_t)(255 - 8 * lane - j);
-        sm.above = above;
-        sm.cnt = c[j];
-      }
-      above += c[j];
-    }
-  }
-  __syncthreads();
-  const uint32_t b_lo = sm.bin * width;
-  rem -= sm.above;
-  const int cnt = sm.cnt;
-  base += b_lo;
-  span_m1 = min(width - 1u, span_m1 - b_lo);
-  for (int j = tid; j < 256; j += NT) sm.hist[j] = 0;
-  __syncthreads();
-  return cnt;
-}
-
-// The cut of the `need` best candidates (by key, higher first) of [0, n):
-// on return every candidate key above [base, base + span_m1] is kept, every
-// one below it dropped, and the first `rem` inside it (by index) are kept.
-// All NT threads call it, each with the min and max key of the candidates it
-// saw (lo/hi; the block combines them), and sm.hist zeroed.
-//
-// Starting from the candidates' [min, max] spreads keys over the bins however
-// their exponents cluster; each pass shrinks the interval 256-fold until one
-// key value is left or the boundary bin is kept whole.
-template <int NT, typename KeyF, typename StateF>
-__device__ void topk_cut(int n, int need, KeyF key, StateF state, TopkSmem<NT>& sm, uint32_t lo, uint32_t hi,
-                         uint32_t& base, uint32_t& span_m1, int& rem) {
-  static_assert(NT >= 256 && NT % 32 == 0 && NT <= 1024, "block shape");
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  base = 0;
-  span_m1 = 0xFFFFFFFFu;
-  rem = need;
-  if (need <= 0) return;
+__device__ __forceinline__ void block_minmax(uint32_t& lo, uint32_t& hi, uint32_t* rmin, uint32_t* rmax) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
     hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
   }
   if (lane == 0) {
-    sm.rmin[warp] = lo;
-    sm.rmax[warp] = hi;
+    rmin[warp] = lo;
+    rmax[warp] = hi;
   }
-  if (tid == 0) sm.cand_n = 0;
   __syncthreads();
-  lo = 0xFFFFFFFFu;
-  hi = 0u;
+  lo = lane < NT / 32 ? rmin[lane] : 0xFFFFFFFFu;
+  hi = lane < NT / 32 ? rmax[lane] : 0u;
   #pragma unroll
-  for (int w = 0; w < NT / 32; ++w) {
-    lo = min(lo, sm.rmin[w]);
-    hi = max(hi, sm.rmax[w]);
-  }
-  base = lo;
-  span_m1 = hi - lo;
-  auto full = [&](int i, uint32_t& kk) {
-    if (state(i) != ST_CAND) return false;
-    kk = key(i);
-    return true;
-  };
-  const int cnt = span_m1 > 0 ? interval_pass<NT>(n, full, base, span_m1, rem, sm) : 0;
-  if (span_m1 == 0 || cnt == rem) return;
-  if (cnt <= kCandCap) {
-    // gather the boundary bin's keys, then narrow on them alone
-    for (int i = tid; i < n; i += NT) {
-      if (state(i) != ST_CAND) continue;
-      const uint32_t kk = key(i);
-      if (kk >= base && kk - base <= span_m1) sm.cand_key[atomicAdd(&sm.cand_n, 1)] = kk;
-    }
-    __syncthreads();
-    const int m = sm.cand_n;
-    auto small = [&](int i, uint32_t& kk) {
-      kk = sm.cand_key[i];
-      return true;
-    };
-    #pragma unroll 1
-    for (int pass = 0; pass < 4 && span_m1 > 0; ++pass)
-      if (interval_pass<NT>(m, small, base, span_m1, rem, sm) == rem) break;
-  } else {
-    #pragma unroll 1
-    for (int pass = 0; pass < 4 && span_m1 > 0; ++pass)
-      if (interval_pass<NT>(n, full, base, span_m1, rem, sm) == rem) break;
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
   }
 }
 
-// Places the kept elements of [0, n) given the cut: emit(slot, index) is
-// called once per kept element, slot = its rank in the ascending list.  Warp
-// w walks the w-th contiguous segment of the vector 32 elements at a time.
-// All NT threads call it.
-template <int NT, typename KeyF, typename StateF, typename EmitF>
-__device__ void topk_place(int n, int need, uint32_t base, uint32_t span_m1, int rem, KeyF key, StateF state,
-                           EmitF emit, TopkSmem<NT>& sm) {
-  constexpr int NW = NT / 32;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t top = base + span_m1;            // inclusive upper end
-  const int seg = ((n + NW * 32 - 1) / (NW * 32)) * 32;
-  const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
-  auto flags = [&](int i, bool& gt, bool& eq) {
-    gt = false;
-    eq = false;
-    if (i >= s1) return;
-    const uint8_t st = state(i);
-    if (st == ST_FORCED) {
-      gt = true;
-    } else if (st == ST_CAND && need > 0) {
-      const uint32_t kk = key(i);
-      gt = kk > top;
-      eq = kk >= base && kk <= top;
+// Within one warp: the bin of a 256-bin histogram H where the count from the
+// top reaches rem (1 <= rem <= total), the count above that bin and the
+// bin's own count, returned to every lane.
+__device__ __forceinline__ void warp_find_bin(const int* H, int rem, int& bin, int& above, int& cnt) {
+  const int lane = threadIdx.x & 31;
+  int c[8], sum = 0;
+  #pragma unroll
+  for (int j = 0; j < 8; ++j) {                   // lane owns bins 255-8*lane .. 248-8*lane
+    c[j] = H[255 - 8 * lane - j];
+    sum += c[j];
+  }
+  int incl = sum;
+  #pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int a = incl - sum, b = -1, ab = 0, cb = 0;
+  #pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (a < rem && a + c[j] >= rem) {
+      b = 255 - 8 * lane - j;
+      ab = a;
+      cb = c[j];
     }
+    a += c[j];
+  }
+  const unsigned who = __ballot_sync(0xffffffffu, b >= 0);
+  const int src = who ? __ffs(who) - 1 : 0;
+  bin = __shfl_sync(0xffffffffu, b, src);
+  above = __shfl_sync(0xffffffffu, ab, src);
+  cnt = __shfl_sync(0xffffffffu, cb, src);
+}
+
+template <int NT>
+struct RegTopkSmem {
+  int hist[3][256];
+  uint32_t rmin[32], rmax[32];
+  int wtot[2][32];
+};
+
+// Writes the forced elements and the `need` candidates of largest key of
+// [0, n) (ties to the lower index) to out, ascending.  n <= NT*KPT; kr as
+// described above (entries of elements >= n are ignored); state(i) is
+// ST_CAND, ST_FORCED (kept, not ranked) or ST_OUT.  All NT threads call it.
+template <int NT, int KPT, typename StateF>
+__device__ void reg_topk(const uint32_t (&kr)[KPT], int n, int need, StateF state, int* out,
+                         RegTopkSmem<NT>& sm) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ibase = warp * KPT * 32 + lane;
+  // the state of key c (recomputed where needed: fewer live registers)
+  auto st = [&](int c) { return ibase + 32 * c < n ? state(ibase + 32 * c) : (uint8_t)ST_OUT; };
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  #pragma unroll
+  for (int c = 0; c < KPT; ++c)
+    if (st(c) == ST_CAND) {
+      lo = min(lo, kr[c]);
+      hi = max(hi, kr[c]);
+    }
+  for (int j = tid; j < 2 * 256; j += NT) (&sm.hist[0][0])[j] = 0;
+  block_minmax<NT>(lo, hi, sm.rmin, sm.rmax);      // its barrier also orders the clearing
+  uint32_t base = lo, span = hi - lo;
+  int rem = need;
+  if (need <= 0) span = 0;
+  #pragma unroll 1
+  for (int pass = 0; pass < 5 && span > 0; ++pass) {
+    int* H = sm.hist[pass % 3];
+    const int sh = max(0, 24 - __clz(span));
+    #pragma unroll
+    for (int c = 0; c < KPT; ++c) {
+      const uint32_t kk = kr[c];
+      if (st(c) == ST_CAND && kk >= base && kk - base <= span) atomicAdd(&H[(kk - base) >> sh], 1);
+    }
+    __syncthreads();
+    int bin, above, cnt;
+    warp_find_bin(H, rem, bin, above, cnt);
+    // the histogram of the previous pass: every warp read it before this
+    // pass's barrier, and the pass after next counts into it
+    int* Z = sm.hist[(pass + 2) % 3];
+    for (int j = tid; j < 256; j += NT) Z[j] = 0;
+    const uint32_t b_lo = (uint32_t)bin << sh;
+    rem -= above;
+    base += b_lo;
+    span = min((1u << sh) - 1u, span - b_lo);
+    if (cnt == rem) break;                          // the whole bin is kept
+  }
+  // placement: kept above the interval (gt) or inside it (eq), per row of 32
+  const uint32_t top = base + span;
+  auto rows = [&](int c, unsigned& gm, unsigned& em) {
+    const uint8_t s = st(c);
+    const bool in = need > 0 && s == ST_CAND;
+    const uint32_t kk = kr[c];
+    gm = __ballot_sync(0xffffffffu, s == ST_FORCED || (in && kk > top));
+    em = __ballot_sync(0xffffffffu, in && kk >= base && kk <= top);
   };
   int gt_w = 0, eq_w = 0;
-  for (int c = s0; c < s1; c += 32) {
-    bool g, e;
-    flags(c + lane, g, e);
-    gt_w += __popc(__ballot_sync(0xffffffffu, g));
-    eq_w += __popc(__ballot_sync(0xffffffffu, e));
+  #pragma unroll
+  for (int c = 0; c < KPT; ++c) {
+    unsigned gm, em;
+    rows(c, gm, em);
+    gt_w += __popc(gm);
+    eq_w += __popc(em);
   }
   if (lane == 0) {
     sm.wtot[0][warp] = gt_w;
     sm.wtot[1][warp] = eq_w;
   }
   __syncthreads();
-  int gt_b = 0, eq_b = 0;
-  for (int w = 0; w < warp; ++w) {
-    gt_b += sm.wtot[0][w];
-    eq_b += sm.wtot[1][w];
+  int gt_b = lane < warp ? sm.wtot[0][lane] : 0;   // the warps before this one
+  int eq_b = lane < warp ? sm.wtot[1][lane] : 0;
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    gt_b += __shfl_xor_sync(0xffffffffu, gt_b, o);
+    eq_b += __shfl_xor_sync(0xffffffffu, eq_b, o);
   }
-  const unsigned lt = (1u << lane) - 1u;
-  for (int c = s0; c < s1; c += 32) {
-    bool g, e;
-    flags(c + lane, g, e);
-    const unsigned gm = __ballot_sync(0xffffffffu, g), em = __ballot_sync(0xffffffffu, e);
+  const unsigned lt = (1u << lane) - 1u, me = 1u << lane;
+  #pragma unroll
+  for (int c = 0; c < KPT; ++c) {
+    unsigned gm, em;
+    rows(c, gm, em);
     const int gb = gt_b + __popc(gm & lt), eb = eq_b + __popc(em & lt);
-    if (g || (e && eb < rem)) emit(gb + min(eb, rem), c + lane);
+    if ((gm & me) || ((em & me) && eb < rem)) out[gb + min(eb, rem)] = ibase + 32 * c;
     gt_b += __popc(gm);
     eq_b += __popc(em);
   }
-}
-
-// Writes the forced elements and the `need` best candidates of [0, n) (ties
-// to the lower index) to out, ascending.
-template <int NT, typename KeyF, typename StateF>
-__device__ void radix_topk(int n, int need, KeyF key, StateF state, int* out, TopkSmem<NT>& sm,
-                           uint32_t lo, uint32_t hi) {
-  uint32_t base, span_m1;
-  int rem;
-  topk_cut<NT>(n, need, key, state, sm, lo, hi, base, span_m1, rem);
-  topk_place<NT>(n, need, base, span_m1, rem, key, state, [&](int slot, int i) { out[slot] = i; }, sm);
 }
 
 }  // namespace bc

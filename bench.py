@@ -144,6 +144,31 @@ class Clocks:
                 "power_w_max": max((num(p[2]) or 0) for p in inside)}
 
 
+def record_traffic(csv_path, key="k_gemv_gateup", kernel="k_gemv", source="gemv.cu"):
+    """Writes profiles/traffic.json from an ncu raw-page CSV export
+    (`ncu -i rep --page raw --csv`) of `--only-kernel gemv_gateup`: the mean
+    DRAM bytes read + written per captured launch of `kernel`, stamped with
+    the kernel source's hash so a later change of the source voids it."""
+    import csv
+    rows = list(csv.reader(open(csv_path)))
+    hdr, units = rows[0], rows[1]
+    scale = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    ir, iw, ik = hdr.index("dram__bytes_read.sum"), hdr.index("dram__bytes_write.sum"), hdr.index("Kernel Name")
+    per = [float(r[ir].replace(",", "")) * scale[units[ir]] + float(r[iw].replace(",", "")) * scale[units[iw]]
+           for r in rows[2:] if r[ik].split("(")[0].split("<")[0].split()[-1] == kernel]
+    if not per:
+        raise SystemExit(f"no {kernel} launches in {csv_path}")
+    src = os.path.join(ROOT, "activation_kv_sparsity_b200", "csrc", source)
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    d = json.load(open(p)) if os.path.exists(p) else {}
+    d[key] = {"source": source, "source_sha": sha, "dram_bytes_per_launch": round(sum(per) / len(per)),
+              "launches": len(per), "capture": "ncu --set full --clock-control none -k regex:k_gemv -s 3 -c 1 "
+                                               "python bench.py --only-kernel gemv_gateup --steps 3 --warmup 3"}
+    json.dump(d, open(p, "w"), indent=1)
+    return d[key]
+
+
 def traffic_record(kernel):
     """DRAM bytes per launch from the committed ncu summary, valid only while
     the kernel source is unchanged since the capture."""
@@ -660,9 +685,14 @@ def main():
                     choices=["dense", "act", "kv", "both"])
     ap.add_argument("--timeline", choices=("dense", "act", "kv", "both"),
                     help="per-site cost of one step in this mode at the first --contexts value")
+    ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
+                    help="write profiles/traffic.json from an ncu raw CSV of --only-kernel gemv_gateup")
     ap.add_argument("--only-kernel", choices=("gemv_gateup", "gemv_gateup_dense", "attention"),
                     help="time one kernel alone on a small case (profiler captures)")
     args = ap.parse_args()
+    if args.record_traffic:
+        print(json.dumps(record_traffic(args.record_traffic)))
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

@@ -118,6 +118,34 @@ def test_graph_steps_equal_direct_steps(tiny, mode):
         assert torch.equal(a, b), (mode, i)
 
 
+@pytest.mark.parametrize("edge", [32768, 131072])
+def test_graph_steps_across_page_select_variants(tiny, edge):
+    """Across 2048 -> 2049 pages (32768 tokens) the one-CTA page select moves
+    from 2 to 4 keys a thread, across 8192 -> 8193 pages (131072 tokens) to
+    the cluster: a new graph is captured for the new variant and the steps
+    still equal direct launches bit for bit, with exact page sets."""
+    cfg = tiny["cfg"]
+    n0 = edge - 12
+    k, v = make_kv(cfg, n0, seed=5, device=DEV)
+    outs = {}
+    for graphs in (False, True):
+        m = bc.Model(cfg, tiny["wd"], edge + 32)
+        m.append(k, v)
+        m.set_graphs(graphs)
+        logits = torch.empty(cfg["vocab"], device=DEV)
+        seq = []
+        for tok in tokens(24, cfg["vocab"], seed=13):
+            m.step(tok, "kv", logits, **KW)
+            seq.append(logits.clone())
+        torch.cuda.synchronize()
+        tr = gpu_traces(m, cfg["n_layers"], True)
+        check_selection_exact(tr, KW["rp"], KW["rkv"], KW["sinks"], KW["recent"], False, True)
+        outs[graphs] = seq
+        m.close()
+    for i, (a, b) in enumerate(zip(outs[False], outs[True])):
+        assert torch.equal(a, b), i
+
+
 def _meta(m, cfg, max_ctx):
     Pmax = -(-max_ctx // 16)
     return m.meta_pool.view(torch.bfloat16).view(cfg["n_layers"], cfg["n_kv_heads"], Pmax, 2, cfg["head_dim"])

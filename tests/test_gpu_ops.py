@@ -66,13 +66,15 @@ def test_gemv_is_deterministic():
 @pytest.mark.parametrize("n", [1, 7, 100, 1024, 1792, 4096, 14336, 16384])
 def test_select_topk_exact(n):
     g = _gen(n)
-    for trial in range(3):
+    for trial in range(4):
         v = torch.randn(n, generator=g)
         if trial == 1:
             v = torch.round(v * 4) / 4            # many ties
         if trial == 2:
             v = torch.zeros(n)                    # all tied
             v[:: 3] = 1.0
+        if trial == 3:
+            v = 1.0 + 1e-4 * v                    # narrow range: crowded bins
         vd = v.to(DEV)
         for k in sorted({1, max(1, n // 3), max(1, math.ceil(0.7 * n - 1e-9)), n}):
             idx = torch.full((k,), -1, dtype=torch.int32, device=DEV)
