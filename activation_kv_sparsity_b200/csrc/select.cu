@@ -46,7 +46,7 @@ constexpr int kSelSlice = kMaxSelect / kSelCluster;   // largest slice
 
 struct SelClusterSmem {
   int hist[2][256];
-  int ghist[256];
+  alignas(16) int ghist[256];
   int red[32];
   uint32_t rmin[32], rmax[32];
   uint32_t lo, hi;
@@ -100,34 +100,13 @@ __device__ void cluster_topk(const uint32_t* s_key, int s0, int ns, int need, St
       sm.hist[(pass + 1) & 1][tid] = 0;
     }
     __syncthreads();
-    if (warp == 0) {
-      int c[8], sum = 0;
-      #pragma unroll
-      for (int j = 0; j < 8; ++j) {              // lane owns bins 255-8*lane .. 248-8*lane
-        c[j] = sm.ghist[255 - 8 * lane - j];
-        sum += c[j];
-      }
-      int incl = sum;
-      #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      int above = incl - sum;
-      #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (above < rem && above + c[j] >= rem) {
-          sm.bin = (uint32_t)(255 - 8 * lane - j);
-          sm.above = above;
-          sm.cnt = c[j];
-        }
-        above += c[j];
-      }
-    }
-    __syncthreads();
-    const uint32_t b_lo = sm.bin << sh;
-    rem -= sm.above;
-    const int cnt = sm.cnt;
+    // every warp finds the boundary bin itself (the next pass writes ghist
+    // only after the next cluster barrier, which every warp reaches after
+    // reading it)
+    int bin, above, cnt;
+    warp_find_bin(sm.ghist, rem, bin, above, cnt);
+    const uint32_t b_lo = (uint32_t)bin << sh;
+    rem -= above;
     base += b_lo;
     span_m1 = min((1u << sh) - 1u, span_m1 - b_lo);
     if (cnt == rem) break;                        // the whole bin is kept
@@ -234,7 +213,9 @@ __global__ void __launch_bounds__(kSelClThreads, 1) k_select(SelectArgs a) {
 // Vectors up to kSelOneCta elements: one CTA ranks the whole vector with its
 // keys in registers (a cluster's barriers cost more than they save at this
 // size).  Warp w loads the elements (w*KPT + c)*32 + lane, c < KPT: rows of
-// 32 consecutive elements, all KPT rows in flight together.
+// 32 consecutive elements, all KPT rows in flight together.  (256 threads
+// with 16 keys each ran faster alone but slower inside the step: 7.5 against
+// 5.8 us per selection.)
 constexpr int kSelOneCta = 8192;
 constexpr int kSelThreads1 = 1024;
 
@@ -387,8 +368,34 @@ __global__ void __launch_bounds__(kPageThreads, GMAX <= 4 ? 2 : 1) k_pages(PageA
   const int h = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int sub = lane / LPP, cl = lane % LPP;
+  const __nv_bfloat16* mbase = a.meta + (size_t)h * a.Pmax * 2 * HD;
+  float* scores = a.scores + (size_t)h * a.Pmax;
+  const int p_cta = blockIdx.x * a.rounds * PPR;
+  auto page_of = [&](int round, int it) { return p_cta + round * PPR + (it * (kPageThreads / 32) + warp) * PPW + sub; };
+  auto load_one = [&](int p, uint4& mn, uint4& mx) {
+    const __nv_bfloat16* mp = mbase + (size_t)p * 2 * HD + cl * 8;
+    mn = ld_stream(mp);
+    mx = ld_stream(mp + HD);
+  };
+  auto load_round = [&](int round, uint4* mn, uint4* mx, int p_end) {
+    #pragma unroll
+    for (int it = 0; it < STEPS; ++it) {
+      const int p = page_of(round, it);
+      mn[it] = make_uint4(0, 0, 0, 0);
+      mx[it] = mn[it];
+      if (round < a.rounds && p < p_end) load_one(p, mn[it], mx[it]);
+    }
+  };
+  // The bounds do not depend on the previous kernel except those of the last
+  // page, which the q/k/v epilogue rewrites as it appends: load the first
+  // round's others before waiting for it.
+  uint4 mna[STEPS], mxa[STEPS], mnb[STEPS], mxb[STEPS];
+  load_round(0, mna, mxa, a.P - 1);
   pdl_wait();
   pdl_trigger();
+  #pragma unroll
+  for (int it = 0; it < STEPS; ++it)
+    if (a.rounds > 0 && page_of(0, it) == a.P - 1) load_one(a.P - 1, mna[it], mxa[it]);
   float qv[GMAX][8];   // [head][channel]
   #pragma unroll
   for (int g = 0; g < GMAX; ++g) {
@@ -401,23 +408,6 @@ __global__ void __launch_bounds__(kPageThreads, GMAX <= 4 ? 2 : 1) k_pages(PageA
     qv[g][0] = q0.x; qv[g][1] = q0.y; qv[g][2] = q0.z; qv[g][3] = q0.w;
     qv[g][4] = q1.x; qv[g][5] = q1.y; qv[g][6] = q1.z; qv[g][7] = q1.w;
   }
-  const __nv_bfloat16* mbase = a.meta + (size_t)h * a.Pmax * 2 * HD;
-  float* scores = a.scores + (size_t)h * a.Pmax;
-  const int p_cta = blockIdx.x * a.rounds * PPR;
-  auto page_of = [&](int round, int it) { return p_cta + round * PPR + (it * (kPageThreads / 32) + warp) * PPW + sub; };
-  auto load_round = [&](int round, uint4* mn, uint4* mx) {
-    #pragma unroll
-    for (int it = 0; it < STEPS; ++it) {
-      const int p = page_of(round, it);
-      mn[it] = make_uint4(0, 0, 0, 0);
-      mx[it] = mn[it];
-      if (round < a.rounds && p < a.P) {
-        const __nv_bfloat16* mp = mbase + (size_t)p * 2 * HD + cl * 8;
-        mn[it] = ld_stream(mp);
-        mx[it] = ld_stream(mp + HD);
-      }
-    }
-  };
   auto score_round = [&](int round, const uint4* mn, const uint4* mx) {
     #pragma unroll
     for (int it = 0; it < STEPS; ++it) {
@@ -426,20 +416,19 @@ __global__ void __launch_bounds__(kPageThreads, GMAX <= 4 ? 2 : 1) k_pages(PageA
       if (p < a.P && cl == 0) scores[p] = best;
     }
   };
-  uint4 mna[STEPS], mxa[STEPS], mnb[STEPS], mxb[STEPS];
-  load_round(0, mna, mxa);
   for (int r = 0; r < a.rounds; r += 2) {
-    load_round(r + 1, mnb, mxb);
+    load_round(r + 1, mnb, mxb, a.P);
     score_round(r, mna, mxa);
     if (r + 1 >= a.rounds) break;
-    load_round(r + 2, mna, mxa);
+    load_round(r + 2, mna, mxa, a.P);
     score_round(r + 1, mnb, mxb);
   }
 }
 
 // Page select above 8192 pages: one cluster per kv head; CTA r ranks the
 // r-th slice of the head's page scores.  Forced pages (sinks, recent) are
-// kept and not ranked.  (One CTA with 16 keys a thread measured slower.)
+// kept and not ranked.  (One 1024-thread CTA with 16 keys a thread measured
+// slower.)
 __global__ void __launch_bounds__(kSelClThreads, 1) k_page_select(PageArgs a) {
   __shared__ uint32_t s_key[kSelSlice];
   __shared__ SelClusterSmem sm;

@@ -26,40 +26,35 @@ namespace bc {
 
 enum : uint8_t { ST_OUT = 0, ST_CAND = 1, ST_FORCED = 2 };
 
-// Block-wide min of lo and max of hi, returned to every thread (one barrier).
+// Block-wide min of lo and max of hi, returned to every thread (one barrier;
+// warp reductions in hardware).
 template <int NT>
 __device__ __forceinline__ void block_minmax(uint32_t& lo, uint32_t& hi, uint32_t* rmin, uint32_t* rmax) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-  }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
   if (lane == 0) {
     rmin[warp] = lo;
     rmax[warp] = hi;
   }
   __syncthreads();
-  lo = lane < NT / 32 ? rmin[lane] : 0xFFFFFFFFu;
-  hi = lane < NT / 32 ? rmax[lane] : 0u;
-  #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-  }
+  lo = __reduce_min_sync(0xffffffffu, lane < NT / 32 ? rmin[lane] : 0xFFFFFFFFu);
+  hi = __reduce_max_sync(0xffffffffu, lane < NT / 32 ? rmax[lane] : 0u);
 }
 
-// Within one warp: the bin of a 256-bin histogram H where the count from the
-// top reaches rem (1 <= rem <= total), the count above that bin and the
-// bin's own count, returned to every lane.
+// Within one warp: the bin of a 256-bin histogram H (16-byte aligned) where
+// the count from the top reaches rem (1 <= rem <= total), the count above
+// that bin and the bin's own count, returned to every lane.  Lane l reads
+// its 8 bins 255-8l .. 248-8l as two 16-byte loads: the warp's loads are
+// conflict-free, which matters because every warp of the block runs this.
 __device__ __forceinline__ void warp_find_bin(const int* H, int rem, int& bin, int& above, int& cnt) {
   const int lane = threadIdx.x & 31;
-  int c[8], sum = 0;
+  const int4* H4 = reinterpret_cast<const int4*>(H) + 2 * (31 - lane);
+  const int4 v0 = H4[0], v1 = H4[1];             // bins 248-8l .. 251-8l, 252-8l .. 255-8l
+  const int c[8] = {v1.w, v1.z, v1.y, v1.x, v0.w, v0.z, v0.y, v0.x};
+  int sum = 0;
   #pragma unroll
-  for (int j = 0; j < 8; ++j) {                   // lane owns bins 255-8*lane .. 248-8*lane
-    c[j] = H[255 - 8 * lane - j];
-    sum += c[j];
-  }
+  for (int j = 0; j < 8; ++j) sum += c[j];
   int incl = sum;
   #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -85,7 +80,7 @@ __device__ __forceinline__ void warp_find_bin(const int* H, int rem, int& bin, i
 
 template <int NT>
 struct RegTopkSmem {
-  int hist[3][256];
+  alignas(16) int hist[3][256];
   uint32_t rmin[32], rmax[32];
   int wtot[2][32];
 };
@@ -157,13 +152,9 @@ __device__ void reg_topk(const uint32_t (&kr)[KPT], int n, int need, StateF stat
     sm.wtot[1][warp] = eq_w;
   }
   __syncthreads();
-  int gt_b = lane < warp ? sm.wtot[0][lane] : 0;   // the warps before this one
-  int eq_b = lane < warp ? sm.wtot[1][lane] : 0;
-  #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    gt_b += __shfl_xor_sync(0xffffffffu, gt_b, o);
-    eq_b += __shfl_xor_sync(0xffffffffu, eq_b, o);
-  }
+  // the warps before this one
+  int gt_b = (int)__reduce_add_sync(0xffffffffu, lane < warp ? (unsigned)sm.wtot[0][lane] : 0u);
+  int eq_b = (int)__reduce_add_sync(0xffffffffu, lane < warp ? (unsigned)sm.wtot[1][lane] : 0u);
   const unsigned lt = (1u << lane) - 1u, me = 1u << lane;
   #pragma unroll
   for (int c = 0; c < KPT; ++c) {
