@@ -30,7 +30,18 @@ Readings of what the pages leave open (each is a choice, stated once):
 * rotary embedding: rotate-half pairs (i, i + hd/2), inv_freq_i = theta^(-2i/hd),
   no frequency rescaling; cached keys are already rotated;
 * RMSNorm x / sqrt(mean(x^2) + eps) * g; SwiGLU silu(gate) * up;
-  the LM head is dense in every mode.
+  the LM head is dense in every mode;
+* once-after-prefill selection (the pages' own KV mode, SnapKV-style: an
+  attention-scored choice made once after prefill, README "Timing and
+  quality on a GPU"; SnapKV is listed on the mlsanity page): a window of
+  observation queries per query head (the last prompt positions' queries,
+  post-rotary; synthetic here) votes for the cached tokens with its softmax
+  attention over the whole prefix (scale 1/sqrt(hd)); a page's score is the
+  attention mass its valid tokens receive from all observation queries of
+  the kv head's group; the same page rule as above keeps the sinks, the
+  recent pages and the best scored others; the kept pages are frozen, and
+  every decode step afterwards attends over them plus every page begun
+  after the selection ("snap" mode, dense projections).
 
 Arithmetic: fp64 throughout, on bf16 weights and KV widened exactly.
 """
@@ -140,6 +151,38 @@ def page_select(scores: np.ndarray, rkv: float, sinks: int, recent: int) -> np.n
     return np.array(sorted(F | set(rest[:K - len(F)])), dtype=np.int64)
 
 
+def snap_scores(q_obs: np.ndarray, keys: np.ndarray, n_tok: int, page: int) -> np.ndarray:
+    """Once-after-prefill page scores of one kv head: the softmax attention
+    mass that the observation queries q_obs [Q][hd] put on each page's valid
+    tokens (keys [>= n_tok][hd]), summed over the queries.  Returns [P]; the
+    scores sum to Q."""
+    s = q_obs @ keys[:n_tok].T / math.sqrt(q_obs.shape[-1])
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p /= p.sum(axis=1, keepdims=True)
+    mass = p.sum(axis=0)
+    P = -(-n_tok // page)
+    padded = np.zeros(P * page)
+    padded[:n_tok] = mass
+    return padded.reshape(P, page).sum(axis=1)
+
+
+def snap_select(cfg, cache: "Cache", q_obs, rkv: float, sinks: int, recent: int):
+    """The once-after-prefill selection over the cache's n tokens.  q_obs
+    [L][W][Hq][hd] float64 (post-rotary).  Returns ({(layer, kv head):
+    ascending kept pages}, {(layer, kv head): page scores}, P at selection)."""
+    L, Hq, Hkv, hd = cfg["n_layers"], cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"]
+    G, page, n = Hq // Hkv, cfg["page"], cache.n
+    kept, scores = {}, {}
+    for l in range(L):
+        for h in range(Hkv):
+            qs = np.asarray(q_obs[l][:, h * G:(h + 1) * G], dtype=np.float64).reshape(-1, hd)
+            sc = snap_scores(qs, bf16_to_f64(cache.k[l, h, :n]), n, page)
+            scores[(l, h)] = sc
+            kept[(l, h)] = page_select(sc, rkv, sinks, recent)
+    return kept, scores, -(-n // page)
+
+
 def attention(q: np.ndarray, keys: np.ndarray, values: np.ndarray, tok: np.ndarray):
     """Softmax attention of the G query heads q [G][hd] over the tokens
     ``tok`` of one kv head; scale 1/sqrt(hd).  Returns [G][hd]."""
@@ -183,12 +226,12 @@ class Cache:
         self.n += c
 
 
-MODES = ("dense", "act", "kv", "both")
+MODES = ("dense", "act", "kv", "both", "snap")
 
 
 def decode_step(cfg, w, cache: Cache, token: int, mode: str, rp=1.0, rkv=1.0,
                 sinks=1, recent=16, forced=None, kv_round=True, layers=None,
-                x_in=None, trace=None):
+                x_in=None, trace=None, snap=None):
     """One decode step at position cache.n.  Appends the token's k, v.
 
     w: dict of bf16 bit arrays in the layouts of ``synth.make_weights``.
@@ -198,6 +241,8 @@ def decode_step(cfg, w, cache: Cache, token: int, mode: str, rp=1.0, rkv=1.0,
     layers: optional range of layers to run (the rest are skipped and the
         logits are not computed); x_in: residual stream entering the first of
         them (default: the token's embedding row).
+    snap: for mode 'snap', (kept pages per (layer, kv head), P at the
+        selection) as returned by ``snap_select``.
     trace: optional dict that receives every intermediate per layer.
     Returns the logits [V] (or the residual stream when ``layers`` is given).
     """
@@ -243,7 +288,13 @@ def decode_step(cfg, w, cache: Cache, token: int, mode: str, rp=1.0, rkv=1.0,
             if k_new is not None:
                 keys[pos], vals[pos] = k_new[h], v_new[h]
             qg = q[h * G:(h + 1) * G]
-            if kvsel:
+            if mode == "snap":
+                kept, p_snap = snap
+                sel = np.array(sorted(set(int(p) for p in kept[(l, h)]) | set(range(p_snap, P))),
+                               dtype=np.int64)
+                tok = np.concatenate([np.arange(p * page, min((p + 1) * page, n_tok)) for p in sel])
+                pages_l.append(sel)
+            elif kvsel:
                 kmin, kmax = page_bounds(keys, n_tok, page)
                 sc = page_scores(qg, kmin, kmax)
                 if (l, "pages", h) in forced:

@@ -334,3 +334,89 @@ def test_appended_kv_is_rounded_to_bf16(tiny):
     od.decode_step(cfg, w, cache, 7, "dense", trace=trace)
     np.testing.assert_array_equal(cache.k[0, :, N_CTX], od.f64_to_bf16(trace[0]["k"]))
     assert cache.n == N_CTX + 1
+
+
+# ----------------------------------------------------------------- once-after-prefill selection
+
+def test_snap_scores_match_sdpa_page_masses():
+    """Page scores are the attention mass per page: SDPA with one-hot page
+    indicators as values gives each query's mass per page directly; a
+    ragged last page counts only its valid tokens."""
+    Q, hd, n, page = 12, 32, 77, 16
+    q = RNG.standard_normal((Q, hd))
+    k = RNG.standard_normal((n + 5, hd)) * 1.5
+    got = od.snap_scores(q, k, n, page)
+    P = -(-n // page)
+    onehot = np.zeros((n, P))
+    onehot[np.arange(n), np.arange(n) // page] = 1.0
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, None], torch.from_numpy(k[:n])[None, None],
+        torch.from_numpy(onehot)[None, None])[0, 0].numpy().sum(axis=0)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+    assert got.shape == (P,) and abs(got.sum() - Q) < 1e-12
+
+
+def test_snap_scores_follow_a_planted_key():
+    """A key aligned with every observation query draws almost all the
+    mass to its page."""
+    Q, hd, n, page = 8, 64, 160, 16
+    u = RNG.standard_normal(hd)
+    u /= np.linalg.norm(u)
+    q = np.outer(np.ones(Q), u) * 4.0 + 0.01 * RNG.standard_normal((Q, hd))
+    k = RNG.standard_normal((n, hd)) * 0.1
+    k[83] = 40.0 * u                              # logit 4 * 40 / 8 = 20 above the rest
+    sc = od.snap_scores(q, k, n, page)
+    assert int(np.argmax(sc)) == 83 // page and sc[83 // page] > 0.99 * Q
+
+
+def test_snap_select_keeps_forced_and_best(tiny):
+    cfg, _, w, kb, vb = tiny
+    cache = od.Cache(cfg, N_CTX + 4)
+    cache.extend(kb[:, :, :N_CTX], vb[:, :, :N_CTX])
+    rng = np.random.default_rng(3)
+    q_obs = rng.standard_normal((cfg["n_layers"], 4, cfg["n_heads"], cfg["head_dim"]))
+    kept, scores, P = od.snap_select(cfg, cache, q_obs, 0.3, 1, 2)
+    assert P == -(-N_CTX // cfg["page"])
+    for (l, h), sel in kept.items():
+        F = od.forced_pages(P, 1, 2)
+        assert F <= set(sel.tolist())
+        K = max(len(F), math.ceil(0.3 * P - 1e-9))
+        assert len(sel) == K
+        rest = [p for p in range(P) if p not in F]
+        best = sorted(rest, key=lambda p: (-scores[(l, h)][p], p))[:K - len(F)]
+        assert set(best) == set(sel.tolist()) - F
+
+
+def test_snap_mode_all_pages_is_dense_and_forced_only_is_the_window(tiny):
+    """Keeping every page reproduces dense exactly; keeping only the forced
+    pages, at a step inside the last selected page, is the kv mode's window
+    (K = |F|) exactly."""
+    cfg, _, w, kb, vb = tiny
+    tok = tokens(6, cfg["vocab"], seed=5)[5]
+    n = N_CTX - 3                                   # the step stays inside the last page
+    P = -(-n // cfg["page"])
+    everything = {(l, h): np.arange(P) for l in range(cfg["n_layers"]) for h in range(cfg["n_kv_heads"])}
+    dense, _ = _oracle(cfg, w, kb, vb, n, tok, "dense")
+    snap, _ = _oracle(cfg, w, kb, vb, n, tok, "snap", snap=(everything, P))
+    np.testing.assert_array_equal(snap, dense)
+    F = np.array(sorted(od.forced_pages(P, 1, 2)))
+    only_forced = {key: F for key in everything}
+    snap_f, ts = _oracle(cfg, w, kb, vb, n, tok, "snap", snap=(only_forced, P))
+    window, tw = _oracle(cfg, w, kb, vb, n, tok, "kv", rkv=1e-6, sinks=1, recent=2)
+    np.testing.assert_array_equal(snap_f, window)
+    for l in range(cfg["n_layers"]):
+        for a, b in zip(ts[l]["pages"], tw[l]["pages"]):
+            np.testing.assert_array_equal(a, b)
+
+
+def test_snap_mode_takes_pages_begun_after_the_selection(tiny):
+    """A step that opens a new page attends over the frozen pages plus the
+    new one."""
+    cfg, _, w, kb, vb = tiny
+    n = 18 * cfg["page"]                            # the step's token opens page 18
+    P = n // cfg["page"]
+    frozen = {(l, h): np.array([0, 5, P - 1]) for l in range(cfg["n_layers"]) for h in range(cfg["n_kv_heads"])}
+    _, tr = _oracle(cfg, w, kb, vb, n, tokens(2, cfg["vocab"], seed=9)[1], "snap", snap=(frozen, P))
+    for l in range(cfg["n_layers"]):
+        for sel in tr[l]["pages"]:
+            np.testing.assert_array_equal(sel, [0, 5, P - 1, P])
