@@ -19,11 +19,11 @@ _lib = C.CDLL(LIB_PATH)
 
 # ------------------------------------------------------------------ enums
 BC_OK, BC_EINVAL, BC_ENOMEM, BC_ECAPACITY, BC_ECUDA, BC_ETIMEOUT = range(6)
-BC_DENSE, BC_ACT, BC_KV, BC_BOTH = range(4)
-MODES = {"dense": BC_DENSE, "act": BC_ACT, "kv": BC_KV, "both": BC_BOTH}
+BC_DENSE, BC_ACT, BC_KV, BC_BOTH, BC_SNAP = range(5)
+MODES = {"dense": BC_DENSE, "act": BC_ACT, "kv": BC_KV, "both": BC_BOTH, "snap": BC_SNAP}
 (BC_TRACE_XN, BC_TRACE_SEL_QKV, BC_TRACE_Q, BC_TRACE_ATTN, BC_TRACE_SEL_O, BC_TRACE_XN2,
  BC_TRACE_SEL_GU, BC_TRACE_H, BC_TRACE_SEL_D, BC_TRACE_X, BC_TRACE_PAGE_SCORES, BC_TRACE_PAGES,
- BC_TRACE_QKV) = range(13)
+ BC_TRACE_QKV, BC_TRACE_SNAP_SCORES, BC_TRACE_SNAP_PAGES) = range(15)
 
 
 class bc_config(C.Structure):
@@ -59,6 +59,7 @@ _SIGS = {
     "bc_launch_count": (C.c_longlong, [_P]),
     "bc_kv_reset": (C.c_int, [_P, C.c_int]),
     "bc_kv_append": (C.c_int, [_P, _P, _P, C.c_int]),
+    "bc_kv_snap_select": (C.c_int, [_P, _P, C.c_int, C.c_float, C.c_int, C.c_int]),
     "bc_decode_step": (C.c_int, [_P, C.c_int, C.c_int, C.c_float, C.c_float, C.c_int, C.c_int, C.c_int, _P]),
     "bc_decode_step_host": (C.c_int, [_P, C.c_int, C.c_int, C.c_float, C.c_float, C.c_int, C.c_int, C.c_int, _P]),
     "bc_trace": (C.c_int, [_P, C.c_int, C.c_int, C.POINTER(_P), C.POINTER(C.c_int), C.POINTER(C.c_int)]),
@@ -169,6 +170,13 @@ class Model:
         check(bc_kv_append(self.h, C.c_void_p(k.data_ptr()), C.c_void_p(v.data_ptr()), k.shape[2]),
               "bc_kv_append")
 
+    def snap_select(self, q_obs, rkv, sinks=1, recent=16):
+        """Once-after-prefill page selection; q_obs: f32 device tensor
+        [L][n_obs][Hq][hd] of rotated observation queries."""
+        q_obs = q_obs.contiguous()
+        check(bc_kv_snap_select(self.h, C.c_void_p(q_obs.data_ptr()), q_obs.shape[1], rkv, sinks, recent),
+              "bc_kv_snap_select")
+
     def step(self, token: int, mode: str, logits, rp=1.0, rkv=1.0, sinks=1, recent=16):
         check(bc_decode_step(self.h, int(token), MODES[mode], rp, rkv, sinks, recent, self.c.page,
                              C.c_void_p(logits.data_ptr())), "bc_decode_step")
@@ -183,7 +191,8 @@ class Model:
         ptr, cnt, stride = C.c_void_p(), C.c_int(), C.c_int()
         check(bc_trace(self.h, layer, kind, C.byref(ptr), C.byref(cnt), C.byref(stride)), "bc_trace")
         off = ptr.value - self.workspace.data_ptr()
-        is_int = kind in (BC_TRACE_SEL_QKV, BC_TRACE_SEL_O, BC_TRACE_SEL_GU, BC_TRACE_SEL_D, BC_TRACE_PAGES)
+        is_int = kind in (BC_TRACE_SEL_QKV, BC_TRACE_SEL_O, BC_TRACE_SEL_GU, BC_TRACE_SEL_D, BC_TRACE_PAGES,
+                          BC_TRACE_SNAP_PAGES)
         dt = torch.int32 if is_int else torch.float32
         if stride.value:
             rows = self.cfg["n_kv_heads"]

@@ -79,6 +79,8 @@ struct Layout {
   size_t x, xf, logits, xn, qkv, q, attn, xn2, gu, h, xo;    // f32 (per-layer ones are [L][..])
   size_t sel_qkv, sel_o, sel_gu, sel_d;                         // int32 [L][..]
   size_t pscore, pages;                                         // [L][Hkv][Pmax]
+  size_t snap_scores, snap_pages;                               // [L][Hkv][Pmax]
+  size_t snap_part, snap_stats;                                 // float2 [Hkv][chunks][Q], [Hkv][Q]
   size_t part_o, part_ml, gemv_part, counters;
   size_t total;
   int nqkv, hq, Pmax, max_dout;
@@ -118,6 +120,10 @@ static Layout make_layout(const bc_config* c) {
   y.sel_d = take(4 * L * f);
   y.pscore = take(4 * L * c->n_kv_heads * (size_t)y.Pmax);
   y.pages = take(4 * L * c->n_kv_heads * (size_t)y.Pmax);
+  y.snap_scores = take(4 * L * c->n_kv_heads * (size_t)y.Pmax);
+  y.snap_pages = take(4 * L * c->n_kv_heads * (size_t)y.Pmax);
+  y.snap_part = take(8 * (size_t)c->n_kv_heads * snap_chunks(c->max_ctx) * kSnapMaxQ);
+  y.snap_stats = take(8 * (size_t)c->n_kv_heads * kSnapMaxQ);
   y.part_o = take(4 * (size_t)c->n_heads * kMaxSplits * c->head_dim);
   y.part_ml = take(4 * (size_t)c->n_heads * kMaxSplits * 2);
   y.gemv_part = take(4 * (size_t)kGemvMaxContrib * y.max_dout);
@@ -165,6 +171,10 @@ struct bc_model {
   bool last_act;       // the last step ranked activations (XN, XN2, H traces valid)
   // CUDA graphs of the step, one per step configuration
   bool use_graphs;
+  // the once-after-prefill selection: valid until the cache is appended to
+  // in bulk or reset; P and K at the selection
+  bool snap_valid;
+  int snap_P, snap_K;
   cudaStream_t cap_stream;                 // private stream the steps are captured on
   std::vector<struct StepGraph*> graphs;
 };
@@ -245,6 +255,8 @@ extern "C" bc_status bc_model_create(const bc_config* cfg, const bc_weights* w, 
   m->last_P = m->last_K = 0;
   m->last_act = false;
   m->use_graphs = true;
+  m->snap_valid = false;
+  m->snap_P = m->snap_K = 0;
   m->cap_stream = nullptr;
   cudaError_t e = cudaMemsetAsync(m->ws + lay.counters, 0, counter_bytes(cfg, lay), m->stream);
   if (e != cudaSuccess) {
@@ -283,6 +295,49 @@ extern "C" bc_status bc_kv_reset(bc_model* m, int n_ctx) {
   if (!m) return fail(BC_EINVAL, "null model");
   if (n_ctx < 0 || n_ctx > m->n) return fail(BC_EINVAL, "reset to %d outside [0, %d]", n_ctx, m->n);
   m->n = n_ctx;
+  m->snap_valid = false;
+  return BC_OK;
+}
+
+extern "C" bc_status bc_kv_snap_select(bc_model* m, const float* q_obs, int n_obs, float rkv, int sinks,
+                                       int recent) {
+  if (!m || !q_obs) return fail(BC_EINVAL, "null argument");
+  const bc_config& c = m->cfg;
+  const Layout& y = m->lay;
+  const int G = c.n_heads / c.n_kv_heads, Hkv = c.n_kv_heads, L = c.n_layers;
+  if (n_obs < 1 || n_obs * G > kSnapMaxQ)
+    return fail(BC_EINVAL, "n_obs %d outside [1, %d]", n_obs, kSnapMaxQ / G);
+  if (!(rkv > 0.f && rkv <= 1.f)) return fail(BC_EINVAL, "rkv %g outside (0, 1]", rkv);
+  if (sinks < 0 || recent < 1) return fail(BC_EINVAL, "sinks must be >= 0 and recent >= 1");
+  if (m->n < 1) return fail(BC_EINVAL, "the cache holds no tokens");
+  const int n = m->n, P = (n + kPage - 1) / kPage, Pmax = y.Pmax;
+  const int sink_end = std::min(sinks, P), rec_begin = std::max(P - recent, 0);
+  const int n_forced = sink_end + (P - std::max(rec_begin, sink_end));
+  const int K = std::max(n_forced, (int)std::min<double>(P, ceil((double)rkv * P - 1e-9)));
+  const size_t kv_layer = (size_t)Hkv * Pmax * 2 * kPage * c.head_dim;
+  m->snap_valid = false;
+  for (int l = 0; l < L; ++l) {
+    SnapArgs sa;
+    sa.q_obs = q_obs + (size_t)l * n_obs * c.n_heads * c.head_dim;
+    sa.kv = m->kv + l * kv_layer;
+    sa.Hkv = Hkv;
+    sa.G = G;
+    sa.hd = c.head_dim;
+    sa.Pmax = Pmax;
+    sa.n_obs = n_obs;
+    sa.n_tok = n;
+    sa.part = at<float2>(m, y.snap_part);
+    sa.stats = at<float2>(m, y.snap_stats);
+    sa.scores = at<float>(m, y.snap_scores) + (size_t)l * Hkv * Pmax;
+    BC_CUDA(launch_snap_scores(sa, m->stream, true), "snap page scores");
+    PageArgs pa{nullptr, nullptr, Hkv, G, c.head_dim, Pmax, P, K, sinks, recent, 0, sa.scores,
+                at<int>(m, y.snap_pages) + (size_t)l * Hkv * Pmax, nullptr};
+    BC_CUDA(launch_page_select(pa, m->stream, true), "snap page select");
+  }
+  m->launches += 4LL * L;
+  m->snap_valid = true;
+  m->snap_P = P;
+  m->snap_K = K;
   return BC_OK;
 }
 
@@ -307,6 +362,7 @@ extern "C" bc_status bc_kv_append(bc_model* m, const void* k, const void* v, int
   BC_CUDA(launch_kv_append(a, m->stream, true), "bc_kv_append");
   m->launches += 2;
   m->n += n_tokens;
+  m->snap_valid = false;
   return BC_OK;
 }
 
@@ -318,7 +374,9 @@ static int keep_count(float ratio, int n) {
 static bc_status check_step(const bc_model* m, bc_mode mode, float rp, float rkv, int sinks,
                             int recent, int page) {
   if (!m) return fail(BC_EINVAL, "null model");
-  if (mode < BC_DENSE || mode > BC_BOTH) return fail(BC_EINVAL, "bad mode %d", (int)mode);
+  if (mode < BC_DENSE || mode > BC_SNAP) return fail(BC_EINVAL, "bad mode %d", (int)mode);
+  if (mode == BC_SNAP && !m->snap_valid)
+    return fail(BC_EINVAL, "snap mode needs a selection (bc_kv_snap_select) since the last append or reset");
   if (page != m->cfg.page) return fail(BC_EINVAL, "page %d differs from the model's %d", page, m->cfg.page);
   if (!(rp > 0.f && rp <= 1.f)) return fail(BC_EINVAL, "rp %g outside (0, 1]", rp);
   if (!(rkv > 0.f && rkv <= 1.f)) return fail(BC_EINVAL, "rkv %g outside (0, 1]", rkv);
@@ -403,6 +461,7 @@ static bool record(std::vector<NodeRec>* rec, cudaStream_t st, int kind, int lay
 // Per-step values every mode derives from the position.
 struct StepShape {
   int pos, n_tok, P, K, splits, pps;
+  int list_len, tail0;      // attention page list: listed entries, then pages tail0, tail0+1, ...
   int k_qkv, k_o, k_gu, k_d;
 };
 
@@ -415,11 +474,19 @@ static StepShape step_shape(const bc_model* m, bc_mode mode, float rp, float rkv
   sh.n_tok = sh.pos + 1;
   sh.P = (sh.n_tok + kPage - 1) / kPage;
   sh.K = sh.P;
+  sh.list_len = 0;
+  sh.tail0 = 0;
+  if (mode == BC_SNAP) {
+    sh.K = m->snap_K + std::max(0, sh.P - m->snap_P);
+    sh.list_len = m->snap_K;
+    sh.tail0 = m->snap_P;
+  }
   if (kvs) {
     const int sink_end = std::min(sinks, sh.P), rec_begin = std::max(sh.P - recent, 0);
     const int n_forced = sink_end + (sh.P - std::max(rec_begin, sink_end));
     const int want = (int)std::min<double>(sh.P, ceil((double)rkv * sh.P - 1e-9));
     sh.K = std::max(n_forced, want);
+    sh.list_len = sh.K;
   }
   attn_plan(sh.K, c.n_kv_heads, m->sms, &sh.splits, &sh.pps);
   sh.k_qkv = act ? keep_count(rp, c.hidden) : c.hidden;
@@ -540,7 +607,9 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
     AttnArgs aa;
     aa.q = q;
     aa.kv = kvl;
-    aa.pages = kvs ? pages : nullptr;
+    aa.pages = kvs ? pages : mode == BC_SNAP ? at<int>(m, y.snap_pages) + (size_t)l * Hkv * Pmax : nullptr;
+    aa.list_len = sh.list_len;
+    aa.tail0 = sh.tail0;
     aa.Hkv = Hkv;
     aa.G = G;
     aa.hd = hd;
@@ -658,6 +727,8 @@ static cudaError_t launch_step_graph(bc_model* m, StepGraph* g, int token, const
         break;
       case NK_ATTN:
         r.args.a.n_pages = sh.K;
+        r.args.a.list_len = sh.list_len;
+        r.args.a.tail0 = sh.tail0;
         r.args.a.n_tok = sh.n_tok;
         r.args.a.splits = sh.splits;
         r.args.a.pages_per_split = sh.pps;
@@ -766,6 +837,12 @@ extern "C" bc_status bc_trace(const bc_model* m, int layer, bc_trace_kind kind, 
     case BC_TRACE_PAGES:
       off = y.pages + 4ull * layer * c.n_kv_heads * y.Pmax; n = m->last_K; st = y.Pmax; break;
     case BC_TRACE_QKV: off = y.qkv + 4ull * layer * y.nqkv; n = y.nqkv; break;
+    case BC_TRACE_SNAP_SCORES:
+      off = y.snap_scores + 4ull * layer * c.n_kv_heads * y.Pmax; n = m->snap_valid ? m->snap_P : 0; st = y.Pmax;
+      break;
+    case BC_TRACE_SNAP_PAGES:
+      off = y.snap_pages + 4ull * layer * c.n_kv_heads * y.Pmax; n = m->snap_valid ? m->snap_K : 0; st = y.Pmax;
+      break;
     default: return fail(BC_EINVAL, "bad trace kind %d", (int)kind);
   }
   *ptr = m->ws + off;
@@ -846,6 +923,8 @@ extern "C" bc_status bc_attention(const float* q, const void* kv, int n_kv_heads
   a.Pmax = Pmax;
   a.n_pages = n_pages;
   a.n_tok = n_tok;
+  a.list_len = n_pages;
+  a.tail0 = 0;
   attn_plan(n_pages, n_kv_heads, device_sms(), &a.splits, &a.pages_per_split);
   char* sc = static_cast<char*>(scratch);
   const size_t o_bytes = align256(4ull * nq * kMaxSplits * head_dim);

@@ -20,6 +20,10 @@
 // unchanged.  Value fragments are transposed in registers with movmatrix;
 // each lane ends with its head row's output over the same dims.
 //
+// A listed slice may end in an implicit run: entries from list_len on are
+// the pages tail0, tail0 + 1, ... (the pages begun after a once-after-prefill
+// selection).
+//
 // Partials (m, l, o) per (query head, split) use base-2 logits.  The last
 // CTA of each kv head to finish (an atomic ticket, no spinning) merges them:
 // o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, summing in split order.
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn(AttnArgs a) {
   // load; the window moves on by 32 entries long before they are needed.
   auto entry = [&](int jj) {
     const int i = i_begin + warp + kAttnWarps * jj;
-    return i < i_end ? plist[i] : 0;
+    return i < i_end ? (i < a.list_len ? plist[i] : a.tail0 + (i - a.list_len)) : 0;
   };
   int win0 = 0, win1 = 0, base = 0;
   if (plist) {

@@ -13,6 +13,9 @@
 // form per mode: the rows of the kept channels of every projection, the LM
 // head, the valid tokens of the kept pages, the key bounds of every page
 // (kv modes), the append, norm gains, the embedding row and the logits.
+// BC_SNAP reads the pages a once-after-prefill selection made at this
+// context kept, plus a page the step's token opens, and no bounds; its paper
+// form is the KV branch's.
 #include "../../include/bytecross.h"
 
 #include <math.h>
@@ -29,11 +32,12 @@ extern "C" bc_status bc_byte_account(const bc_config* c, bc_mode mode, float rp_
   if (c->n_layers < 1 || c->hidden < 1 || c->intermediate < 1 || c->n_heads < 1 || c->n_kv_heads < 1 ||
       c->head_dim < 1 || c->vocab < 1 || page < 1 || n_ctx < 0 || sinks < 0 || recent < 1)
     return BC_EINVAL;
-  if (mode < BC_DENSE || mode > BC_BOTH) return BC_EINVAL;
+  if (mode < BC_DENSE || mode > BC_SNAP) return BC_EINVAL;
   const double rp = rp_f, rkv = rkv_f;
   if (!(rp > 0 && rp <= 1) || !(rkv > 0 && rkv <= 1)) return BC_EINVAL;
   const bool act = mode == BC_ACT || mode == BC_BOTH;
   const bool kvs = mode == BC_KV || mode == BC_BOTH;
+  const bool snap = mode == BC_SNAP;
   const double L = c->n_layers, d = c->hidden, f = c->intermediate;
   const double hq = (double)c->n_heads * c->head_dim, hkv = (double)c->n_kv_heads * c->head_dim;
   const double hd = c->head_dim, V = c->vocab;
@@ -46,7 +50,7 @@ extern "C" bc_status bc_byte_account(const bc_config* c, bc_mode mode, float rp_
   out->head_bytes = 2 * V * d;
   out->kv_bytes_per_token = 2 * L * 2 * hkv;
   out->dense_bytes = out->weight_bytes + out->head_bytes + n * out->kv_bytes_per_token;
-  const double erp = act ? rp : 1.0, erkv = kvs ? rkv : 1.0;
+  const double erp = act ? rp : 1.0, erkv = (kvs || snap) ? rkv : 1.0;
   out->saved_bytes = (1 - erp) * out->weight_bytes + (1 - erkv) * n * out->kv_bytes_per_token;
   out->bound = out->dense_bytes / (out->dense_bytes - out->saved_bytes);
   const double den = (1 - rkv) * 2 * hkv;
@@ -57,13 +61,18 @@ extern "C" bc_status bc_byte_account(const bc_config* c, bc_mode mode, float rp_
   const long long Hkv = c->n_kv_heads;
   const long long n_tok = n_ctx + 1;
   const long long P = (n_tok + page - 1) / page;
+  auto kept = [&](long long pages) {
+    const long long sink_end = std::min<long long>(sinks, pages);
+    const long long rec_begin = std::max<long long>(pages - recent, 0);
+    const long long forced = sink_end + (pages - std::max(rec_begin, sink_end));
+    const long long want = std::min<long long>(pages, (long long)ceil(rkv * (double)pages - 1e-9));
+    return std::max(forced, want);
+  };
   long long K = P;
-  if (kvs) {
-    const long long sink_end = std::min<long long>(sinks, P);
-    const long long rec_begin = std::max<long long>(P - recent, 0);
-    const long long forced = sink_end + (P - std::max(rec_begin, sink_end));
-    const long long want = std::min<long long>(P, (long long)ceil(rkv * (double)P - 1e-9));
-    K = std::max(forced, want);
+  if (kvs) K = kept(P);
+  if (snap) {
+    const long long P_sel = (std::max<long long>(n_ctx, 1) + page - 1) / page;
+    K = kept(P_sel) + std::max<long long>(0, P - P_sel);
   }
   const long long qkv_cols = (long long)(hq + 2 * hkv);
   const long long kq = act ? keep_rows(rp, c->hidden) : c->hidden;
@@ -74,7 +83,7 @@ extern "C" bc_status bc_byte_account(const bc_config* c, bc_mode mode, float rp_
   out->impl_head_bytes = 2 * V * d;
   // the last page (partial, always kept: it is recent) holds n_tok - (P-1)*page tokens
   const long long last = n_tok - (P - 1) * page;
-  const long long tokens_read = kvs ? (K - 1) * page + last : n_tok;
+  const long long tokens_read = (kvs || snap) ? (K - 1) * page + last : n_tok;
   out->impl_kv_read_bytes = L * (double)Hkv * (double)tokens_read * 2 * hd * 2;
   out->impl_meta_read_bytes = kvs ? L * (double)Hkv * (double)P * 2 * hd * 2 : 0.0;
   out->impl_kv_write_bytes = L * (double)Hkv * (2 * hd * 2 + 2 * hd * 2);

@@ -91,12 +91,26 @@ int page_select_variant(int P);
 int page_rounds(int P, int hd, int Hkv, int sms);
 dim3 pages_grid(const PageArgs& a);
 
+// ------------------------------------------------------------------ once-after-prefill page scores
+constexpr int kSnapMaxQ = 128;    // observation queries per kv head (n_obs * G)
+struct SnapArgs {
+  const float* q_obs;             // this layer's observation queries [n_obs][Hq][hd], post-rotary
+  const __nv_bfloat16* kv;        // this layer's pages [Hkv][Pmax][2][16][hd]
+  int Hkv, G, hd, Pmax, n_obs, n_tok;
+  float2* part;                   // [Hkv][snap_chunks(n_tok)][Q] per-chunk (max, sum), base 2
+  float2* stats;                  // [Hkv][Q] (max, sum) over all n_tok tokens
+  float* scores;                  // [Hkv][Pmax] page scores (attention mass)
+};
+int snap_chunks(int n_tok);
+cudaError_t launch_snap_scores(const SnapArgs& a, cudaStream_t st, bool pdl);
+
 // ------------------------------------------------------------------ attention
 struct AttnArgs {
   const float* q;                 // [Hkv*G][hd]
   const __nv_bfloat16* kv;        // layer pages [Hkv][Pmax][2][16][hd]
   const int* pages;               // [Hkv][Pmax] or nullptr (pages 0..n_pages-1)
   int Hkv, G, hd, Pmax, n_pages, n_tok;
+  int list_len, tail0;            // entries >= list_len are pages tail0, tail0+1, ... (not listed)
   int splits, pages_per_split;
   float* part_o;                  // [Hkv*G][kMaxSplits][hd]
   float* part_ml;                 // [Hkv*G][kMaxSplits][2]

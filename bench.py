@@ -42,7 +42,15 @@ HEAD_MODE, HEAD_CTX = "both", 32768
 KEEP = dict(rp=0.5, rkv=0.3, sinks=1, recent=16)
 CONTEXTS = (131072, 65536, 32768, 8192, 2048)         # descending: every cell sees pristine synthetic KV
 MODE_KW = {"dense": dict(), "act": dict(rp=0.5), "kv": dict(rkv=0.3, sinks=1, recent=16),
-           "both": dict(rp=0.5, rkv=0.3, sinks=1, recent=16)}
+           "both": dict(rp=0.5, rkv=0.3, sinks=1, recent=16),
+           # the pages' KV window baseline: the kv mode with no scored pages
+           # (K = |F|: the sink page and the 16 recent pages)
+           "window": dict(rkv=1e-6, sinks=1, recent=16),
+           # the pages' own KV mode: one selection after prefill (16 observation
+           # positions per query head), then steps over the frozen pages
+           "snap": dict(rkv=0.3, sinks=1, recent=16)}
+SNAP_OBS = 16
+LIB_MODE = {"window": "kv"}                          # bench cells that run a library mode
 CROSS_PAIRS = ((0.7, 0.3), (0.5, 0.3), (0.5, 0.5))
 
 
@@ -188,7 +196,7 @@ def traffic_record(kernel):
 def run_ours(args, rank, ws, local):
     import torch
     import activation_kv_sparsity_b200 as bc
-    from synth import LLAMA_8B, kv_chunks, make_weights
+    from synth import LLAMA_8B, kv_chunks, make_weights, obs_queries
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -208,11 +216,23 @@ def run_ours(args, rank, ws, local):
     clocks = Clocks(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local))
     peak, peak_kind = peaks()
 
+    q_obs = obs_queries(cfg, SNAP_OBS, device=dev) if "snap" in args.modes else None
+    snap_select_ms = {}
+
     def time_cell(mode, n):
         kw = MODE_KW[mode]
+        lib = LIB_MODE.get(mode, mode)
         model.reset(n)
+        if mode == "snap":
+            # the selection is paid once per prefill: timed apart from the steps
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            model.snap_select(q_obs, **kw)
+            s1.record(stream)
+            torch.cuda.synchronize()
+            snap_select_ms[n] = s0.elapsed_time(s1)
         for i in range(warm):
-            model.step(toks[i], mode, logits, **kw)
+            model.step(toks[i], lib, logits, **kw)
         torch.cuda.synchronize()
         barrier(ws)
         l0 = model.launches()
@@ -221,7 +241,7 @@ def run_ours(args, rank, ws, local):
         e0.record(stream)
         h0 = time.perf_counter()
         for i in range(steps):
-            model.step(toks[warm + i], mode, logits, **kw)
+            model.step(toks[warm + i], lib, logits, **kw)
         host_enqueue[(mode, n)] = (time.perf_counter() - h0) * 1e3 / steps
         e1.record(stream)
         torch.cuda.synchronize()
@@ -256,21 +276,30 @@ def run_ours(args, rank, ws, local):
         for mode in args.modes:
             ms, launches = time_cell(mode, n)
             kw = dict(KEEP)
+            kw.update(MODE_KW[mode])
             # the timed steps run at contexts n+warm .. n+warm+steps-1: average their byte accounts
-            accs = [bc.byte_account(cfg, mode, n + warm + i, **kw) for i in range(steps)]
+            accs = [bc.byte_account(cfg, LIB_MODE.get(mode, mode), n + warm + i, **kw) for i in range(steps)]
             acc = dict(accs[0])
             acc["impl_total_bytes"] = sum(a["impl_total_bytes"] for a in accs) / steps
+            if mode == "snap":
+                # the step right after the selection at n, plus every token
+                # appended since (each is read: frozen partial page, new pages)
+                base = bc.byte_account(cfg, "snap", n, **kw)["impl_total_bytes"]
+                tok_bytes = cfg["n_layers"] * cfg["n_kv_heads"] * 2 * cfg["head_dim"] * 2
+                acc["impl_total_bytes"] = base + tok_bytes * (warm + (steps - 1) / 2.0)
             gbs = acc["impl_total_bytes"] / (ms * 1e-3) / 1e9
             cells[(mode, n)] = dict(mode=mode, context=n, ms_per_step=round(ms, 4),
                                     tok_s=round(1000.0 / ms, 2), bytes_per_step=acc["impl_total_bytes"],
                                     gbs=round(gbs, 1), frac_of_measured_peak=round(gbs / peak, 4),
                                     paper_bound=round(acc["bound"], 4), launches_per_step=launches // steps,
                                     host_enqueue_ms=round(host_enqueue[(mode, n)], 4))
+            if mode == "snap":
+                cells[(mode, n)]["selection_ms_once"] = round(snap_select_ms[n], 3)
     for n in contexts:
         if ("dense", n) not in cells:
             continue
         d = cells[("dense", n)]["ms_per_step"]
-        for mode in ("act", "kv", "both"):
+        for mode in ("act", "kv", "both", "window", "snap"):
             if (mode, n) in cells:
                 cells[(mode, n)]["speedup_vs_dense"] = round(d / cells[(mode, n)]["ms_per_step"], 4)
 
@@ -681,8 +710,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--contexts", type=int, nargs="+", default=list(CONTEXTS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--modes", nargs="+", default=["dense", "act", "kv", "both"],
-                    choices=["dense", "act", "kv", "both"])
+    ap.add_argument("--modes", nargs="+", default=["dense", "act", "kv", "both", "window", "snap"],
+                    choices=["dense", "act", "kv", "both", "window", "snap"])
     ap.add_argument("--timeline", choices=("dense", "act", "kv", "both"),
                     help="per-site cost of one step in this mode at the first --contexts value")
     ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",

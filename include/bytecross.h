@@ -45,7 +45,7 @@ typedef enum {
 
 /* Decode modes (ByteCross README, "Timing and quality on a GPU": dense,
  * proj, sel, both). */
-typedef enum { BC_DENSE = 0, BC_ACT = 1, BC_KV = 2, BC_BOTH = 3 } bc_mode;
+typedef enum { BC_DENSE = 0, BC_ACT = 1, BC_KV = 2, BC_BOTH = 3, BC_SNAP = 4 } bc_mode;
 
 /* Model dimensions: the Hugging Face config fields the README's byte account
  * reads ("Quick start"), plus KV capacity and page size.
@@ -134,15 +134,39 @@ BC_API long long bc_launch_count(const bc_model* m);
 
 /* Truncates the cache to its first n_ctx tokens (0 <= n_ctx <= length).
  * Host-only: later appends recompute the bounds of the page they land in
- * from its valid keys, so nothing on the device needs clearing. */
+ * from its valid keys, so nothing on the device needs clearing.  Voids a
+ * once-after-prefill selection. */
 BC_API bc_status bc_kv_reset(bc_model* m, int n_ctx);
 
 /* Appends n_tokens (>= 0) keys and values to every layer and kv head.
  * k, v: device bf16 [L][Hkv][n_tokens][hd], keys already rotated (they stand
  * for what a dense prefill wrote).  Writes the pages and recomputes the key
- * bounds of every page touched.  Async on the model's stream.
+ * bounds of every page touched.  Voids a once-after-prefill selection.
+ * Async on the model's stream.
  * Errors: BC_ECAPACITY if length + n_tokens > max_ctx; BC_EINVAL; BC_ECUDA. */
 BC_API bc_status bc_kv_append(bc_model* m, const void* k, const void* v, int n_tokens);
+
+/* Once-after-prefill page selection over the n = bc_kv_length(m) cached
+ * tokens: the pages' own KV mode (ByteCross README, "Timing and quality on a
+ * GPU": an attention-scored selection made once after prefill, in the
+ * manner of SnapKV).  A window of n_obs observation queries per query head
+ * (the last prompt positions' queries, rotated) votes with its softmax
+ * attention over all n tokens (scale 1/sqrt(hd)); the score of a page of kv
+ * head h is the attention mass its valid tokens receive from the n_obs*G
+ * observation queries of h's group.  With P = ceil(n/page) pages, the same
+ * rule as the KV branch keeps K = clamp(ceil(rkv*P - 1e-9), |F|, P) pages:
+ * the forced first `sinks` and last `recent` pages and the best scored
+ * others (descending, ties: lower page).  The kept lists are frozen: every
+ * later BC_SNAP step attends over them plus every page begun after the
+ * selection, with no per-step scoring.
+ *   q_obs  device f32 [L][n_obs][Hq][hd], read during the call's kernels.
+ *   n_obs  1 <= n_obs and n_obs*G <= 128.
+ * Runs four kernels per layer on the model's stream (not captured in the
+ * step graphs); the selection is voided by bc_kv_append and bc_kv_reset.
+ * Traces: BC_TRACE_SNAP_SCORES, BC_TRACE_SNAP_PAGES.
+ * Errors: BC_EINVAL (no tokens, bad sizes or ratios), BC_ECUDA. */
+BC_API bc_status bc_kv_snap_select(bc_model* m, const float* q_obs, int n_obs, float rkv, int sinks,
+                                   int recent);
 
 /* One decode step at position n = bc_kv_length(m) for input token `token`:
  * embedding row, then per layer RMSNorm -> [act: top-k |x| select] -> q/k/v
@@ -152,7 +176,10 @@ BC_API bc_status bc_kv_append(bc_model* m, const void* k, const void* v, int n_t
  * RMSNorm -> [act: select] -> gate/up GEMV -> SwiGLU -> [act: select] ->
  * down GEMV + residual; then final RMSNorm and the dense LM head.
  *
- *   mode    BC_DENSE, BC_ACT, BC_KV, BC_BOTH
+ *   mode    BC_DENSE, BC_ACT, BC_KV, BC_BOTH, or BC_SNAP: dense projections and
+ *           attention over the pages a bc_kv_snap_select kept plus every
+ *           page begun since (BC_EINVAL without a valid selection; rp, rkv,
+ *           sinks and recent are then not used)
  *   rp      projection keep ratio in (0,1]; per projection input of width
  *           d_in the k = ceil(rp*d_in - 1e-9) channels of largest |x| are
  *           read (ties: lower index).  Ignored unless mode is ACT or BOTH.
@@ -198,11 +225,16 @@ BC_API bc_status bc_decode_step_host(bc_model* m, int token, bc_mode mode, float
  *   BC_TRACE_X         residual stream after the layer          [hidden]
  *   BC_TRACE_PAGE_SCORES f32 [Hkv][stride] (count = P, stride = Pmax)
  *   BC_TRACE_PAGES     int32 [Hkv][stride] kept pages ascending (count = K)
- *   BC_TRACE_QKV       raw q/k/v GEMV output before rotation    [(Hq+2Hkv) hd] */
+ *   BC_TRACE_QKV       raw q/k/v GEMV output before rotation    [(Hq+2Hkv) hd]
+ *   BC_TRACE_SNAP_SCORES f32 [Hkv][stride] page scores of the last
+ *                      once-after-prefill selection (count = its P)
+ *   BC_TRACE_SNAP_PAGES int32 [Hkv][stride] its kept pages, ascending
+ *                      (count = its K) */
 typedef enum {
   BC_TRACE_XN = 0, BC_TRACE_SEL_QKV, BC_TRACE_Q, BC_TRACE_ATTN, BC_TRACE_SEL_O,
   BC_TRACE_XN2, BC_TRACE_SEL_GU, BC_TRACE_H, BC_TRACE_SEL_D, BC_TRACE_X,
-  BC_TRACE_PAGE_SCORES, BC_TRACE_PAGES, BC_TRACE_QKV, BC_TRACE_COUNT
+  BC_TRACE_PAGE_SCORES, BC_TRACE_PAGES, BC_TRACE_QKV, BC_TRACE_SNAP_SCORES, BC_TRACE_SNAP_PAGES,
+  BC_TRACE_COUNT
 } bc_trace_kind;
 
 BC_API bc_status bc_trace(const bc_model* m, int layer, bc_trace_kind kind,
@@ -269,7 +301,10 @@ BC_API bc_status bc_attention(const float* q, const void* kv, int n_kv_heads, in
  * "Usage: The byte account": Equations 1-5, reconstructed so that every
  * printed value is reproduced).  Implementation form: the bytes this
  * library's step at context n_ctx (n_ctx tokens cached, token n_ctx
- * appended) must move in `mode`. */
+ * appended) must move in `mode`.  For BC_SNAP: the step right after a
+ * once-after-prefill selection made at n_ctx with rkv, sinks and recent
+ * (its kept pages plus a page the token opens; no bounds read); its paper
+ * form is the KV branch's. */
 typedef struct {
   /* paper form */
   double weight_bytes;        /* W = 2 L P_l, the seven projections */

@@ -140,10 +140,13 @@ def implementation_bytes(cfg, mode, n, rp=1.0, rkv=1.0, sinks=1, recent=16):
     """Bytes one decode step moves at context n (n tokens cached; the step
     appends token n and attends over n+1), enumerated explicitly.
 
-    mode: 'dense', 'act', 'kv' or 'both'.  Returns a dict of byte counts.
+    mode: 'dense', 'act', 'kv', 'both' or 'snap' (the pages a once-after-
+    prefill selection made at context n kept, plus a page the step's token
+    opens; no bounds are read).  Returns a dict of byte counts.
     """
     act = mode in ("act", "both")
     kv = mode in ("kv", "both")
+    snap = mode == "snap"
     L, d, f = cfg["n_layers"], cfg["hidden"], cfg["intermediate"]
     Hq, Hkv, hd, V, page = (cfg["n_heads"], cfg["n_kv_heads"], cfg["head_dim"],
                             cfg["vocab"], cfg["page"])
@@ -161,6 +164,10 @@ def implementation_bytes(cfg, mode, n, rp=1.0, rkv=1.0, sinks=1, recent=16):
                 # the forced recent pages include the last (partial) page
                 pages = _selected_page_count_tokens(P, K, n_tok, page)
                 out["meta_read"] += P * 2 * hd * BF16
+            elif snap:
+                P_sel = -(-max(n, 1) // page)
+                K_sel, _ = page_keep(P_sel, rkv, sinks, recent)
+                pages = _selected_page_count_tokens(P, K_sel + (P - P_sel), n_tok, page)
             else:
                 pages = n_tok
             out["kv_read"] += pages * 2 * hd * BF16

@@ -15,7 +15,10 @@ Recipe (Llama-style GQA decoder, bf16 storage):
 * planted keys (retrieval check): per (layer, kv head) a seeded unit
   direction u; 8 token positions spread evenly over the non-forced pages get
   the key 8 * sqrt(head_dim) * u;
-* token ids: seeded uniform integers in [0, vocab).
+* token ids: seeded uniform integers in [0, vocab);
+* observation queries (once-after-prefill selection): per layer, window
+  position and query head a vector N(0, 1) in fp32, standing in for the last
+  prompt positions' rotated queries.
 
 The weights are drawn layer by layer and kind by kind in a fixed order, the
 KV cache chunk by chunk (``KV_CHUNK`` tokens), so that the values depend only
@@ -159,6 +162,13 @@ def plant_keys(k: torch.Tensor, positions: list[int], seed: int = 7,
         if first_token <= pos < first_token + c:
             k[:, :, pos - first_token, :] = key
     return k
+
+
+def obs_queries(cfg: dict, n_obs: int, seed: int = 11, device="cpu") -> torch.Tensor:
+    """Observation-window queries f32 [L][n_obs][Hq][hd], N(0, 1)."""
+    g = _gen(seed, device)
+    shape = (cfg["n_layers"], n_obs, cfg["n_heads"], cfg["head_dim"])
+    return torch.randn(shape, generator=g, device=device, dtype=torch.float32)
 
 
 def tokens(n: int, vocab: int, seed: int = 2) -> list[int]:

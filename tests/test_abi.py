@@ -107,7 +107,7 @@ def test_library_bound_and_ff_match_printed():
     assert round(bc.byte_account(m, "both", 0, rp=0.5, rkv=0.3)["n_star_ff"] / 1024, 1) == 60.0
 
 
-@pytest.mark.parametrize("mode", ["dense", "act", "kv", "both"])
+@pytest.mark.parametrize("mode", ["dense", "act", "kv", "both", "snap"])
 @pytest.mark.parametrize("n", [0, 15, 16, 2047, 8191, 32768, 131071])
 @pytest.mark.parametrize("cfg", [TINY, LLAMA_8B], ids=["tiny", "8b"])
 def test_library_implementation_bytes_match_oracle(cfg, mode, n):

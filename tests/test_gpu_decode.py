@@ -65,6 +65,29 @@ def test_tiny_eight_steps(tiny, mode):
     assert len(m) == N_CTX + 8
 
 
+def test_kv_window_baseline(tiny):
+    """The KV window (the pages' window baseline: sinks and recent pages
+    only, no scored pages) is the kv mode with a keep ratio small enough that
+    K = |F|: every head keeps exactly the forced pages, and the step matches
+    the oracle."""
+    cfg = tiny["cfg"]
+    kw = dict(rp=1.0, rkv=1e-6, sinks=1, recent=8)
+    m = _model(tiny)
+    cache = _cache(tiny)
+    logits = torch.empty(cfg["vocab"], device=DEV)
+    for tok in tokens(3, cfg["vocab"], seed=17):
+        m.step(tok, "kv", logits, **kw)
+        torch.cuda.synchronize()
+        tr = gpu_traces(m, cfg["n_layers"], True)
+        P = -(-len(m) // 16)
+        want = np.array(sorted(od.forced_pages(P, kw["sinks"], kw["recent"])))
+        for r in tr:
+            for h in range(r["pages"].shape[0]):
+                np.testing.assert_array_equal(r["pages"][h], want)
+        compare_step(cfg, tiny["wb"], cache, tok, "kv", kw["rp"], kw["rkv"], kw["sinks"], kw["recent"],
+                     to_host(logits), tr)
+
+
 def test_keep_one_is_dense_bit_for_bit(tiny):
     cfg = tiny["cfg"]
     m = _model(tiny)
