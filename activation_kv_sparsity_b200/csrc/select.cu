@@ -51,8 +51,6 @@ struct SelClusterSmem {
   uint32_t rmin[32], rmax[32];
   uint32_t lo, hi;
   int gt_tot, eq_tot;
-  uint32_t bin;
-  int above, cnt;
 };
 
 // Ranks the candidates of a vector split over the cluster: this CTA holds the
