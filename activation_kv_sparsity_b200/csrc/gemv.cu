@@ -17,11 +17,12 @@
 //               initialises the residual stream with it
 //   SWIGLU      v = silu(gate) * up
 //
-// Work split: a column tile of 256 outputs is shared by the CTAs of one or
-// more thread-block clusters, and the tile's k listed rows are cut into one
-// contiguous run per CTA.  Each of a CTA's 8 warps streams every 8th row of
-// its run with 16 rows (8 KiB) in flight, 16 bytes per lane per row; warps are
-// reduced in shared memory.  The CTAs of a cluster then sum their partials
+// Work split: a column tile of TW = 256 outputs (128 when there would be
+// fewer than 24 wide tiles) is shared by the CTAs of one or more thread-block
+// clusters, and the tile's k listed rows are cut into one contiguous run per
+// CTA.  A row segment is TW*2 bytes read by TW/8 lanes at 16 bytes each; a
+// CTA's 8 warps stream its run with 16 row segments per lane in flight;
+// warps are reduced in shared memory.  The CTAs of a cluster then sum their partials
 // through distributed shared memory after a hardware cluster barrier (rank 0
 // reads them in rank order).  A tile split over several clusters adds one
 // stage through global scratch: each cluster's rank 0 writes its partial and
