@@ -69,15 +69,17 @@ __global__ void __launch_bounds__(kSnapThreads) k_snap(SnapArgs a) {
   float tokmass[4] = {0.f, 0.f, 0.f, 0.f};
   for (int q0 = 0; q0 < Q; q0 += kSnapQTile) {
     __syncthreads();                           // keys staged; the previous tile's queries consumed
-    // query tile: query qi = j*G + g is observation j of head h*G + g
+    // query tile: query qi = j*G + g is observation j of head h*G + g;
+    // consecutive threads take consecutive queries of one dimension, so the
+    // dimension-major stores are conflict-free
     for (int idx = tid; idx < kSnapQTile * HD; idx += kSnapThreads) {
-      const int qi = q0 + idx / HD, d = idx % HD;
+      const int ql = idx % kSnapQTile, d = idx / kSnapQTile, qi = q0 + ql;
       float v = 0.f;
       if (qi < Q) {
         const int j = qi / a.G, g = qi % a.G;
         v = a.q_obs[((size_t)j * a.Hkv * a.G + h * a.G + g) * HD + d] * scale;
       }
-      sm.q[d][idx / HD] = v;
+      sm.q[d][ql] = v;
     }
     __syncthreads();
     float acc[4][8];

@@ -592,6 +592,34 @@ def run_kernel_only(args, local):
     g = torch.Generator(device=dev)
     g.manual_seed(0)
     stream = torch.cuda.current_stream(dev)
+    if args.only_kernel == "snap":
+        # the once-after-prefill scorer of 2 layers at 32K context, 16
+        # observation positions (64 queries per kv head): 2 passes over the keys
+        from synth import kv_chunks, make_weights, obs_queries
+        c2 = dict(cfg, n_layers=2)
+        n = 32768
+        w = make_weights(c2, seed=0, device=dev)
+        model = bc.Model(c2, w, n + 8)
+        for k, v in kv_chunks(c2, n, seed=1, device=dev):
+            model.append(k, v)
+        q_obs = obs_queries(c2, 16, device=dev)
+        flops = 2 * 2 * c2["n_layers"] * c2["n_heads"] * 16 * n * c2["head_dim"]   # two passes, 2 per FMA
+
+        def launch():
+            model.snap_select(q_obs, rkv=0.3, sinks=1, recent=16)
+        for _ in range(args.warmup):
+            launch()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(model.stream)
+        for _ in range(args.steps):
+            launch()
+        e1.record(model.stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        return {"kernel": "snap", "ms_per_selection": round(ms, 4), "flops": flops,
+                "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+                "note": "2 layers at 32K, both passes and the page select; fp32 CUDA cores"}
     if args.only_kernel in ("gemv_gateup", "gemv_gateup_dense"):
         d, d_out = cfg["hidden"], 2 * cfg["intermediate"]
         W = (torch.randn(d, d_out, generator=g, device=dev) * 0.02).to(torch.bfloat16)
@@ -716,7 +744,7 @@ def main():
                     help="per-site cost of one step in this mode at the first --contexts value")
     ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
                     help="write profiles/traffic.json from an ncu raw CSV of --only-kernel gemv_gateup")
-    ap.add_argument("--only-kernel", choices=("gemv_gateup", "gemv_gateup_dense", "attention"),
+    ap.add_argument("--only-kernel", choices=("gemv_gateup", "gemv_gateup_dense", "attention", "snap"),
                     help="time one kernel alone on a small case (profiler captures)")
     args = ap.parse_args()
     if args.record_traffic:

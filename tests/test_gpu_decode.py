@@ -344,6 +344,45 @@ def test_llama8b_shape_step(big, mode):
     assert max_rel(to_host(logits), ref) < REL_TOL
 
 
+def test_llama8b_shape_snap_step(big):
+    """The once-after-prefill selection and one snap step at the 8B shape:
+    kept pages exact on the GPU's own scores, hidden states of layers 0, 1,
+    16 and 31 and the logits within 1e-2 of the oracle replaying those
+    pages."""
+    from synth import obs_queries
+    cfg = big["cfg"]
+    sel = dict(rkv=0.3, sinks=1, recent=16)
+    m = bc.Model(cfg, big["wd"], N8 + 16)
+    m.append(big["k"], big["v"])
+    q_obs = obs_queries(cfg, 16, seed=11, device=DEV)
+    m.snap_select(q_obs, **sel)
+    logits = torch.empty(cfg["vocab"], device=DEV)
+    tok = 4242
+    m.step(tok, "snap", logits)
+    torch.cuda.synchronize()
+    kept = {}
+    for l in range(cfg["n_layers"]):
+        sc = m.trace(l, bc.BC_TRACE_SNAP_SCORES).cpu().numpy().astype(np.float64)
+        pg = m.trace(l, bc.BC_TRACE_SNAP_PAGES).cpu().numpy().astype(np.int64)
+        for h in range(cfg["n_kv_heads"]):
+            np.testing.assert_array_equal(od.page_select(sc[h], **sel), pg[h], err_msg=f"layer {l} head {h}")
+            kept[(l, h)] = pg[h]
+    tr = gpu_traces(m, cfg["n_layers"], False)
+    P = N8 // 16
+    cache = od.Cache(cfg, N8 + 1)
+    cache.extend(big["kb"], big["vb"])
+    for l in (0, 1, 16, 31):
+        cache.n = N8
+        x_in = None if l == 0 else tr[l - 1]["x"]
+        x = od.decode_step(cfg, big["wb"], cache, tok, "snap", snap=(kept, P), layers=range(l, l + 1), x_in=x_in)
+        assert max_rel(tr[l]["x"], x) < REL_TOL, l
+    xf = od.rms_norm(tr[-1]["x"], big["wb"]["final_norm"], cfg["rms_eps"])
+    ref = np.concatenate([od.bf16_to_f64(big["wb"]["lm_head"][i:i + 8192]) @ xf
+                          for i in range(0, cfg["vocab"], 8192)])
+    assert max_rel(to_host(logits), ref) < REL_TOL
+    m.close()
+
+
 def test_llama8b_shape_planted_retrieval():
     cfg = LLAMA_8B
     n, sinks, recent, rkv = 4096, 1, 16, 0.3
