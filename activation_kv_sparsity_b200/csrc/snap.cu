@@ -12,13 +12,18 @@
 //   M_q = max_t s_qt,  L_q = sum_t exp(s_qt - M_q)   (t over all n tokens).
 //
 // Three kernels per layer: per-chunk (max, sum) of every query, their merge,
-// and the page masses (logits recomputed).  A CTA takes a chunk of 8 pages
-// (128 tokens) of one kv head and a tile of up to 64 queries; each thread
-// computes a 4-token x 8-query block of logits from keys and queries staged
-// in shared memory dimension-major (one 16-byte read of keys and two of
-// queries per dimension, conflict-free).  Base-2 logits throughout.  This
-// runs once per selection, not per decode step; it is CUDA-core fp32 work
-// (about 1 FMA per query, key element and pass).
+// and the page masses (logits recomputed).  The logits are a dense
+// contraction (queries x keys x hd), so they run on the tensor cores with the
+// attention kernel's operand layout: mma m16n8k16 with 8 observation queries
+// per A block (rows 0-7 their bf16 "hi" parts, rows 8-15 the residues, so the
+// sum of both keeps about 16 bits of the fp32 query) and 8 keys per B block.
+// A CTA takes a chunk of 32 pages of one kv head; each of its 4 warps takes
+// every 4th page, with the next page's keys in flight (lane (g, t) loads dims
+// u*32 + t*8 .. +8 of key rows g and g+8, and the contraction dims are
+// permuted alike in the query fragments).  The query fragments of all blocks
+// are staged once per CTA in shared memory, one 16-byte read per lane, block
+// and k16 step.  Base-2 logits throughout.  It runs once per selection, not
+// per decode step.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -26,122 +31,154 @@
 
 namespace bc {
 
-constexpr int kSnapThreads = 256;
-constexpr int kSnapTok = 8 * kPage;           // tokens per chunk
-constexpr int kSnapQTile = 64;                // queries per tile
-
-template <int HD>
-struct SnapSmem {
-  alignas(16) float k[HD][kSnapTok];         // keys of the chunk, dimension-major
-  alignas(16) float q[HD][kSnapQTile];       // the query tile, dimension-major
-  float mass[8][kSnapTok];                   // pass 1: token mass per query group
-};
+constexpr int kSnapWarps = 4;
+constexpr int kSnapPages = 32;                // pages per chunk (CTA)
+constexpr int kSnapTok = kSnapPages * kPage;  // tokens per chunk
+constexpr int kSnapBlocks = kSnapMaxQ / 8;    // query blocks of 8
 
 // PASS 0: per-chunk (max, sum) of every query.  PASS 1: page masses.
 template <int HD, int PASS>
-__global__ void __launch_bounds__(kSnapThreads) k_snap(SnapArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  SnapSmem<HD>& sm = *reinterpret_cast<SnapSmem<HD>*>(smem_raw);
+__global__ void __launch_bounds__(kSnapWarps * 32, 2) k_snap(SnapArgs a) {
+  constexpr int KSTEPS = HD / 16;
+  constexpr int U4 = HD / 32;                 // 16-byte vectors per lane and key row
+  constexpr int PAGE_ELEMS = 2 * kPage * HD;
+  extern __shared__ __align__(16) uint4 s_qa[];   // [blocks][KSTEPS][32 lanes]
+  __shared__ float s_m[kSnapWarps][kSnapMaxQ], s_l[kSnapWarps][kSnapMaxQ];
   const int chunk = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
-  const int tt = tid & 31, qq = tid >> 5;      // tokens 4*tt .. +4, queries 8*qq .. +8 of the tile
-  const int Q = a.n_obs * a.G;
-  const int t0 = chunk * kSnapTok;
-  const float scale = 1.4426950408889634f * rsqrtf((float)HD);
+  const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int Q = a.n_obs * a.G, NB = (Q + 7) / 8;
+  const float qscale = 1.4426950408889634f * rsqrtf((float)HD);
   pdl_wait();
   pdl_trigger();
 
-  // keys of the chunk's tokens (pages are consecutive), converted to fp32
-  const __nv_bfloat16* head = a.kv + (size_t)h * a.Pmax * 2 * kPage * HD;
-  constexpr int DC = HD / 8;
-  for (int idx = tid; idx < kSnapTok * DC; idx += kSnapThreads) {
-    const int t = idx % kSnapTok, dc = idx / kSnapTok;
-    const int tok = t0 + t;
-    uint4 w = make_uint4(0, 0, 0, 0);
-    if (tok < a.n_tok) {
-      const int page = tok / kPage, slot = tok % kPage;
-      w = *reinterpret_cast<const uint4*>(head + ((size_t)page * 2 * kPage + slot) * HD + dc * 8);
+  // query fragments: block b holds queries 8b .. 8b+7 (query qi = j*G + gg is
+  // observation j of head h*G + gg); lane (g, t) of k-step s takes dims
+  // (s/2)*32 + 4*(s%2) + t*8 + 0..3 of query 8b + g
+  for (int e = tid; e < NB * KSTEPS * 32; e += kSnapWarps * 32) {
+    const int ln = e % 32, s = (e / 32) % KSTEPS, blk = e / (32 * KSTEPS);
+    const int qi = 8 * blk + (ln >> 2), tt = ln & 3;
+    const int d0 = (s / 2) * 32 + 4 * (s % 2) + tt * 8;
+    float q[4] = {0.f, 0.f, 0.f, 0.f};
+    if (qi < Q) {
+      const int j = qi / a.G, gg = qi % a.G;
+      const float* qp = a.q_obs + ((size_t)j * a.Hkv * a.G + h * a.G + gg) * HD + d0;
+      #pragma unroll
+      for (int c = 0; c < 4; ++c) q[c] = qp[c] * qscale;
     }
-    sm.k[dc * 8 + 0][t] = bf16_lo(w.x); sm.k[dc * 8 + 1][t] = bf16_hi(w.x);
-    sm.k[dc * 8 + 2][t] = bf16_lo(w.y); sm.k[dc * 8 + 3][t] = bf16_hi(w.y);
-    sm.k[dc * 8 + 4][t] = bf16_lo(w.z); sm.k[dc * 8 + 5][t] = bf16_hi(w.z);
-    sm.k[dc * 8 + 6][t] = bf16_lo(w.w); sm.k[dc * 8 + 7][t] = bf16_hi(w.w);
+    uint4 f;
+    split2(q[0], q[1], f.x, f.y);
+    split2(q[2], q[3], f.z, f.w);
+    s_qa[e] = f;
   }
-  float tokmass[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int q0 = 0; q0 < Q; q0 += kSnapQTile) {
-    __syncthreads();                           // keys staged; the previous tile's queries consumed
-    // query tile: query qi = j*G + g is observation j of head h*G + g;
-    // consecutive threads take consecutive queries of one dimension, so the
-    // dimension-major stores are conflict-free
-    for (int idx = tid; idx < kSnapQTile * HD; idx += kSnapThreads) {
-      const int ql = idx % kSnapQTile, d = idx / kSnapQTile, qi = q0 + ql;
-      float v = 0.f;
-      if (qi < Q) {
-        const int j = qi / a.G, g = qi % a.G;
-        v = a.q_obs[((size_t)j * a.Hkv * a.G + h * a.G + g) * HD + d] * scale;
+  __syncthreads();
+
+  // per lane: query g of every block, running (max, sum) or its (M, 1/L)
+  float m_run[kSnapBlocks], l_run[kSnapBlocks];
+  #pragma unroll
+  for (int b = 0; b < kSnapBlocks; ++b) {
+    m_run[b] = -INFINITY;
+    l_run[b] = 0.f;
+    if (PASS == 1 && b < NB && 8 * b + g < Q) {
+      const float2 st = a.stats[(size_t)h * Q + 8 * b + g];
+      m_run[b] = st.x;
+      l_run[b] = 1.0f / st.y;
+    }
+  }
+  const __nv_bfloat16* head = a.kv + (size_t)h * a.Pmax * PAGE_ELEMS;
+  const int p0 = chunk * kSnapPages;
+  const int p_end = min(p0 + kSnapPages, (a.n_tok + kPage - 1) / kPage);
+  auto load = [&](int page, uint4* k0, uint4* k1) {
+    const __nv_bfloat16* pk = head + (size_t)page * PAGE_ELEMS + t * 8;
+    #pragma unroll
+    for (int u = 0; u < U4; ++u) {
+      k0[u] = ld_stream(pk + g * HD + 32 * u);
+      k1[u] = ld_stream(pk + (g + 8) * HD + 32 * u);
+    }
+  };
+  auto process = [&](int page, const uint4* k0, const uint4* k1) {
+    const uint32_t* kr0 = reinterpret_cast<const uint32_t*>(k0);
+    const uint32_t* kr1 = reinterpret_cast<const uint32_t*>(k1);
+    const int valid = min(kPage, a.n_tok - page * kPage);
+    const int tok[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
+    float mass = 0.f;
+    #pragma unroll
+    for (int b = 0; b < kSnapBlocks; ++b) {
+      if (b >= NB) break;
+      float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+      #pragma unroll
+      for (int s = 0; s < KSTEPS; ++s) {
+        const uint4 f = s_qa[(b * KSTEPS + s) * 32 + lane];
+        const uint32_t qa[4] = {f.x, f.y, f.z, f.w};
+        mma16816(c0, qa, kr0[2 * s], kr0[2 * s + 1]);
+        mma16816(c1, qa, kr1[2 * s], kr1[2 * s + 1]);
       }
-      sm.q[d][ql] = v;
-    }
-    __syncthreads();
-    float acc[4][8];
-    #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-    #pragma unroll 4
-    for (int d = 0; d < HD; ++d) {
-      const float4 kv = *reinterpret_cast<const float4*>(&sm.k[d][4 * tt]);
-      const float4 qa = *reinterpret_cast<const float4*>(&sm.q[d][8 * qq]);
-      const float4 qb = *reinterpret_cast<const float4*>(&sm.q[d][8 * qq + 4]);
-      const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
-      const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-      #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(kk[i], qv[j], acc[i][j]);
-    }
-    bool tvalid[4];
-    #pragma unroll
-    for (int i = 0; i < 4; ++i) tvalid[i] = t0 + 4 * tt + i < a.n_tok;
-    #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int qi = q0 + 8 * qq + j;
+      const float sc[4] = {c0[0] + c0[2], c0[1] + c0[3], c1[0] + c1[2], c1[1] + c1[3]};
       if (PASS == 0) {
-        // this warp covers all 128 tokens of the chunk for its 8 queries
-        float m = -INFINITY;
+        float mx = -INFINITY;
         #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (tvalid[i]) m = fmaxf(m, acc[i][j]);
+        for (int j = 0; j < 4; ++j)
+          if (tok[j] < valid) mx = fmaxf(mx, sc[j]);
+        const float m_new = fmaxf(m_run[b], mx);
+        float add = 0.f;
         #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float l = 0.f;
+        for (int j = 0; j < 4; ++j)
+          if (tok[j] < valid) add += exp2f(sc[j] - m_new);
+        l_run[b] = (m_run[b] == -INFINITY ? 0.f : l_run[b] * exp2f(m_run[b] - m_new)) + add;
+        m_run[b] = m_new;
+      } else if (8 * b + g < Q) {
         #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (tvalid[i]) l += exp2f(acc[i][j] - m);
-        #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        if (tt == 0 && qi < Q) a.part[((size_t)h * gridDim.x + chunk) * Q + qi] = make_float2(m, l);
-      } else if (qi < Q) {
-        const float2 st = a.stats[(size_t)h * Q + qi];
-        const float inv = 1.0f / st.y;
-        #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (tvalid[i]) tokmass[i] += exp2f(acc[i][j] - st.x) * inv;
+        for (int j = 0; j < 4; ++j)
+          if (tok[j] < valid) mass += exp2f(sc[j] - m_run[b]) * l_run[b];
       }
     }
+    if (PASS == 1) {
+      #pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mass += __shfl_xor_sync(0xffffffffu, mass, o);
+      if (lane == 0) a.scores[(size_t)h * a.Pmax + page] = mass;
+    }
+  };
+  uint4 ka0[U4], ka1[U4], kb0[U4], kb1[U4];
+  int p = p0 + warp;
+  if (p < p_end) load(p, ka0, ka1);
+  while (p < p_end) {
+    int q = p + kSnapWarps;
+    if (q < p_end) load(q, kb0, kb1);
+    process(p, ka0, ka1);
+    p = q;
+    if (p >= p_end) break;
+    q = p + kSnapWarps;
+    if (q < p_end) load(q, ka0, ka1);
+    process(p, kb0, kb1);
+    p = q;
   }
-  if (PASS == 1) {
-    // sum the 8 query groups, then the 16 tokens of each page
+  if (PASS == 0) {
+    // the quad's lanes hold the same query: merge them, then the warps
     #pragma unroll
-    for (int i = 0; i < 4; ++i) sm.mass[qq][4 * tt + i] = tokmass[i];
+    for (int b = 0; b < kSnapBlocks; ++b) {
+      if (b >= NB) break;
+      float m = m_run[b], l = l_run[b];
+      #pragma unroll
+      for (int o = 1; o < 4; o <<= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o), l2 = __shfl_xor_sync(0xffffffffu, l, o);
+        const float mm = fmaxf(m, m2);
+        l = (m == -INFINITY ? 0.f : l * exp2f(m - mm)) + (m2 == -INFINITY ? 0.f : l2 * exp2f(m2 - mm));
+        m = mm;
+      }
+      if (t == 0) {
+        s_m[warp][8 * b + g] = m;
+        s_l[warp][8 * b + g] = l;
+      }
+    }
     __syncthreads();
-    if (tid < kSnapTok) {
-      float v = 0.f;
+    for (int qi = tid; qi < Q; qi += kSnapWarps * 32) {
+      float M = -INFINITY;
       #pragma unroll
-      for (int w = 0; w < 8; ++w) v += sm.mass[w][tid];
+      for (int w = 0; w < kSnapWarps; ++w) M = fmaxf(M, s_m[w][qi]);
+      float L = 0.f;
       #pragma unroll
-      for (int o = kPage / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o, kPage);
-      const int page = (t0 + tid) / kPage;
-      if ((tid % kPage) == 0 && page * kPage < a.n_tok) a.scores[(size_t)h * a.Pmax + page] = v;
+      for (int w = 0; w < kSnapWarps; ++w)
+        if (s_m[w][qi] != -INFINITY) L += s_l[w][qi] * exp2f(s_m[w][qi] - M);
+      a.part[((size_t)h * gridDim.x + chunk) * Q + qi] = make_float2(M, L);
     }
   }
 }
@@ -168,12 +205,15 @@ int snap_chunks(int n_tok) { return (n_tok + kSnapTok - 1) / kSnapTok; }
 
 template <int HD>
 static cudaError_t launch_hd(const SnapArgs& a, cudaStream_t st, bool pdl) {
-  const size_t smem = sizeof(SnapSmem<HD>);
+  constexpr int KSTEPS = HD / 16;
+  const int NB = (a.n_obs * a.G + 7) / 8;
+  const size_t smem = (size_t)NB * KSTEPS * 32 * sizeof(uint4);
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(k_snap<HD, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int max_smem = kSnapBlocks * KSTEPS * 32 * (int)sizeof(uint4);
+    cudaError_t e = cudaFuncSetAttribute(k_snap<HD, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k_snap<HD, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      e = cudaFuncSetAttribute(k_snap<HD, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
@@ -183,7 +223,7 @@ static cudaError_t launch_hd(const SnapArgs& a, cudaStream_t st, bool pdl) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(chunks, a.Hkv);
-  cfg.blockDim = dim3(kSnapThreads);
+  cfg.blockDim = dim3(kSnapWarps * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = attr;

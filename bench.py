@@ -619,7 +619,7 @@ def run_kernel_only(args, local):
         ms = e0.elapsed_time(e1) / args.steps
         return {"kernel": "snap", "ms_per_selection": round(ms, 4), "flops": flops,
                 "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
-                "note": "2 layers at 32K, both passes and the page select; fp32 CUDA cores"}
+                "note": "2 layers at 32K, both passes and the page select; mma.sync m16n8k16, bf16 keys, hi/lo-split queries"}
     if args.only_kernel in ("gemv_gateup", "gemv_gateup_dense"):
         d, d_out = cfg["hidden"], 2 * cfg["intermediate"]
         W = (torch.randn(d, d_out, generator=g, device=dev) * 0.02).to(torch.bfloat16)
