@@ -22,7 +22,8 @@
 // u*32 + t*8 .. +8 of key rows g and g+8, and the contraction dims are
 // permuted alike in the query fragments).  The query fragments of all blocks
 // are staged once per CTA in shared memory, one 16-byte read per lane, block
-// and k16 step.  Base-2 logits throughout.  It runs once per selection, not
+// and k16 step; each key fragment feeds 4 query blocks in turn, so a warp has
+// 8 independent accumulator chains in flight.  Base-2 logits throughout.  It runs once per selection, not
 // per decode step.
 #include "common.cuh"
 #include "kernels.h"
@@ -35,6 +36,7 @@ constexpr int kSnapWarps = 4;
 constexpr int kSnapPages = 32;                // pages per chunk (CTA)
 constexpr int kSnapTok = kSnapPages * kPage;  // tokens per chunk
 constexpr int kSnapBlocks = kSnapMaxQ / 8;    // query blocks of 8
+constexpr int kSnapGrp = 4;                   // blocks per key-fragment pass: 8 independent mma chains
 
 // PASS 0: per-chunk (max, sum) of every query.  PASS 1: page masses.
 template <int HD, int PASS>
@@ -46,7 +48,8 @@ __global__ void __launch_bounds__(kSnapWarps * 32, 2) k_snap(SnapArgs a) {
   __shared__ float s_m[kSnapWarps][kSnapMaxQ], s_l[kSnapWarps][kSnapMaxQ];
   const int chunk = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-  const int Q = a.n_obs * a.G, NB = (Q + 7) / 8;
+  const int Q = a.n_obs * a.G;
+  const int NB = ((Q + 8 * kSnapGrp - 1) / (8 * kSnapGrp)) * kSnapGrp;   // blocks, zero-padded
   const float qscale = 1.4426950408889634f * rsqrtf((float)HD);
   pdl_wait();
   pdl_trigger();
@@ -102,33 +105,44 @@ __global__ void __launch_bounds__(kSnapWarps * 32, 2) k_snap(SnapArgs a) {
     const int tok[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
     float mass = 0.f;
     #pragma unroll
-    for (int b = 0; b < kSnapBlocks; ++b) {
-      if (b >= NB) break;
-      float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int b0 = 0; b0 < kSnapBlocks; b0 += kSnapGrp) {
+      if (b0 >= NB) break;
+      float c[kSnapGrp][2][4];
       #pragma unroll
-      for (int s = 0; s < KSTEPS; ++s) {
-        const uint4 f = s_qa[(b * KSTEPS + s) * 32 + lane];
-        const uint32_t qa[4] = {f.x, f.y, f.z, f.w};
-        mma16816(c0, qa, kr0[2 * s], kr0[2 * s + 1]);
-        mma16816(c1, qa, kr1[2 * s], kr1[2 * s + 1]);
-      }
-      const float sc[4] = {c0[0] + c0[2], c0[1] + c0[3], c1[0] + c1[2], c1[1] + c1[3]};
-      if (PASS == 0) {
-        float mx = -INFINITY;
+      for (int i = 0; i < kSnapGrp; ++i)
         #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (tok[j] < valid) mx = fmaxf(mx, sc[j]);
-        const float m_new = fmaxf(m_run[b], mx);
-        float add = 0.f;
+        for (int r = 0; r < 4; ++r) c[i][0][r] = c[i][1][r] = 0.f;
+      #pragma unroll
+      for (int s = 0; s < KSTEPS; ++s)
         #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (tok[j] < valid) add += exp2f(sc[j] - m_new);
-        l_run[b] = (m_run[b] == -INFINITY ? 0.f : l_run[b] * exp2f(m_run[b] - m_new)) + add;
-        m_run[b] = m_new;
-      } else if (8 * b + g < Q) {
-        #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (tok[j] < valid) mass += exp2f(sc[j] - m_run[b]) * l_run[b];
+        for (int i = 0; i < kSnapGrp; ++i) {
+          const uint4 f = s_qa[((b0 + i) * KSTEPS + s) * 32 + lane];
+          const uint32_t qa[4] = {f.x, f.y, f.z, f.w};
+          mma16816(c[i][0], qa, kr0[2 * s], kr0[2 * s + 1]);
+          mma16816(c[i][1], qa, kr1[2 * s], kr1[2 * s + 1]);
+        }
+      #pragma unroll
+      for (int i = 0; i < kSnapGrp; ++i) {
+        const int b = b0 + i;
+        const float sc[4] = {c[i][0][0] + c[i][0][2], c[i][0][1] + c[i][0][3],
+                             c[i][1][0] + c[i][1][2], c[i][1][1] + c[i][1][3]};
+        if (PASS == 0) {
+          float mx = -INFINITY;
+          #pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (tok[j] < valid) mx = fmaxf(mx, sc[j]);
+          const float m_new = fmaxf(m_run[b], mx);
+          float add = 0.f;
+          #pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (tok[j] < valid) add += exp2f(sc[j] - m_new);
+          l_run[b] = (m_run[b] == -INFINITY ? 0.f : l_run[b] * exp2f(m_run[b] - m_new)) + add;
+          m_run[b] = m_new;
+        } else if (8 * b + g < Q) {
+          #pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (tok[j] < valid) mass += exp2f(sc[j] - m_run[b]) * l_run[b];
+        }
       }
     }
     if (PASS == 1) {
@@ -206,7 +220,8 @@ int snap_chunks(int n_tok) { return (n_tok + kSnapTok - 1) / kSnapTok; }
 template <int HD>
 static cudaError_t launch_hd(const SnapArgs& a, cudaStream_t st, bool pdl) {
   constexpr int KSTEPS = HD / 16;
-  const int NB = (a.n_obs * a.G + 7) / 8;
+  const int Q = a.n_obs * a.G;
+  const int NB = ((Q + 8 * kSnapGrp - 1) / (8 * kSnapGrp)) * kSnapGrp;
   const size_t smem = (size_t)NB * KSTEPS * 32 * sizeof(uint4);
   static bool attr_done = false;
   if (!attr_done) {
@@ -231,7 +246,6 @@ static cudaError_t launch_hd(const SnapArgs& a, cudaStream_t st, bool pdl) {
   cudaError_t e = cudaLaunchKernelEx(&cfg, k_snap<HD, 0>, a);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t c2 = cfg;
-  const int Q = a.n_obs * a.G;
   c2.gridDim = dim3((a.Hkv * Q + 127) / 128);
   c2.blockDim = dim3(128);
   c2.dynamicSmemBytes = 0;
