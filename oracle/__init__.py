@@ -19,4 +19,4 @@ implementation run in fp64; the activation-sparse and KV-selected modes
 against the same implementation with masked projection inputs and per-head
 attention masks; every selection routine against brute force on small inputs.
 """
-from . import byte_account, decoder  # noqa: F401
+from . import batch, byte_account, decoder  # noqa: F401

@@ -18,7 +18,11 @@ Recipe (Llama-style GQA decoder, bf16 storage):
 * token ids: seeded uniform integers in [0, vocab);
 * observation queries (once-after-prefill selection): per layer, window
   position and query head a vector N(0, 1) in fp32, standing in for the last
-  prompt positions' rotated queries.
+  prompt positions' rotated queries;
+* batch activations (batched projection): per sequence a N(0, 1) vector
+  with a share ``BATCH_SHARED`` of its variance common to the batch, so that
+  the sequences' kept channel sets overlap as much as the README's batch
+  example assumes.
 
 The weights are drawn layer by layer and kind by kind in a fixed order, the
 KV cache chunk by chunk (``KV_CHUNK`` tokens), so that the values depend only
@@ -169,6 +173,23 @@ def obs_queries(cfg: dict, n_obs: int, seed: int = 11, device="cpu") -> torch.Te
     g = _gen(seed, device)
     shape = (cfg["n_layers"], n_obs, cfg["n_heads"], cfg["head_dim"])
     return torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+
+
+# Share of each batch activation's variance carried by a component common to
+# the batch: with it the union of four sequences' top-50% channel sets covers
+# about 92% of the channels, the union fraction the ByteCross README's
+# crossover_batch example takes for four sequences ("Usage: The byte account").
+BATCH_SHARED = 0.37
+
+
+def batch_activations(batch: int, d: int, shared: float = BATCH_SHARED, seed: int = 13,
+                      device="cpu") -> torch.Tensor:
+    """Projection inputs of a batch of sequences, f32 [batch][d]:
+    sqrt(shared) * z0 + sqrt(1 - shared) * z_b with z0, z_b ~ N(0, 1)."""
+    g = _gen(seed, device)
+    z0 = torch.randn(1, d, generator=g, device=device, dtype=torch.float32)
+    zb = torch.randn(batch, d, generator=g, device=device, dtype=torch.float32)
+    return math.sqrt(shared) * z0 + math.sqrt(1.0 - shared) * zb
 
 
 def tokens(n: int, vocab: int, seed: int = 2) -> list[int]:
