@@ -67,12 +67,16 @@ _SIGS = {
     "bc_gemv": (C.c_int, [_P, C.c_int, C.c_int, _P, _P, C.c_int, _P, _P, C.c_size_t, _P]),
     "bc_gemv_noalloc_max_dout": (C.c_int, []),
     "bc_gemv_noalloc": (C.c_int, [_P, C.c_int, C.c_int, _P, _P, C.c_int, _P, _P]),
+    "bc_gemv_batch_scratch_bytes": (C.c_size_t, [C.c_int, C.c_int, C.c_int]),
+    "bc_gemv_batch": (C.c_int, [_P, C.c_int, C.c_int, _P, _P, C.c_int, C.c_int, _P, _P, _P, C.c_size_t, _P]),
     "bc_select_topk": (C.c_int, [_P, C.c_int, C.c_int, _P, _P]),
     "bc_attention_scratch_bytes": (C.c_size_t, [C.c_int, C.c_int]),
     "bc_attention": (C.c_int, [_P, _P, C.c_int, C.c_int, C.c_int, C.c_int, _P, C.c_int, C.c_int, _P, _P,
                                C.c_size_t, _P]),
     "bc_byte_account": (C.c_int, [C.POINTER(bc_config), C.c_int, C.c_float, C.c_float, C.c_longlong, C.c_int,
                                   C.c_int, C.c_int, C.POINTER(bc_bytes)]),
+    "bc_crossover_batch": (C.c_int, [C.POINTER(bc_config), C.c_double, C.c_double, C.c_int,
+                                     C.POINTER(C.c_double)]),
     "bc_last_error": (C.c_char_p, []),
     "bc_status_string": (C.c_char_p, [C.c_int]),
 }
@@ -107,6 +111,14 @@ def byte_account(cfg: dict, mode: str, n_ctx: int, rp=1.0, rkv=1.0, sinks=1, rec
     check(bc_byte_account(C.byref(c), MODES[mode], rp, rkv, n_ctx, sinks, recent, c.page, C.byref(out)),
           "bc_byte_account")
     return {name: getattr(out, name) for name, _ in bc_bytes._fields_}
+
+
+def crossover_batch(cfg: dict, union_keep: float, rkv: float, batch: int) -> float:
+    """bc_crossover_batch: the batch byte crossover, in tokens."""
+    c = config(cfg, 1)
+    out = C.c_double()
+    check(bc_crossover_batch(C.byref(c), union_keep, rkv, batch, C.byref(out)), "bc_crossover_batch")
+    return out.value
 
 
 def _stream_ptr(stream):
@@ -219,6 +231,19 @@ def gemv_noalloc(W, x, idx, y, stream=None):
     check(bc_gemv_noalloc(C.c_void_p(W.data_ptr()), d_in, d_out, C.c_void_p(x.data_ptr()),
                           C.c_void_p(idx.data_ptr()) if idx is not None else None, k, C.c_void_p(y.data_ptr()),
                           _stream_ptr(stream)), "bc_gemv_noalloc")
+
+
+def gemv_batch(W, x, idx, y, scratch, n_union=None, stream=None):
+    """bc_gemv_batch: x [B][d_in] f32, idx [B][k] int32 (or None for all
+    channels), y [B][d_out] f32, n_union an int32 tensor of one element or None."""
+    d_in, d_out = W.shape
+    B = x.shape[0]
+    k = d_in if idx is None else idx.shape[1]
+    check(bc_gemv_batch(C.c_void_p(W.data_ptr()), d_in, d_out, C.c_void_p(x.data_ptr()),
+                        C.c_void_p(idx.data_ptr()) if idx is not None else None, k, B,
+                        C.c_void_p(y.data_ptr()), C.c_void_p(n_union.data_ptr()) if n_union is not None else None,
+                        C.c_void_p(scratch.data_ptr()), scratch.numel() * scratch.element_size(),
+                        _stream_ptr(stream)), "bc_gemv_batch")
 
 
 def select_topk(v, k, idx, stream=None):

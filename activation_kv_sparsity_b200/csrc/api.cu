@@ -882,6 +882,37 @@ extern "C" bc_status bc_gemv(const void* W, int d_in, int d_out, const float* x,
   return BC_OK;
 }
 
+extern "C" size_t bc_gemv_batch_scratch_bytes(int d_in, int d_out, int batch) {
+  if (d_in < 1 || d_in > kMaxSelect || d_out < kColTile || d_out % kColTile || batch < 1 || batch > kBatchMax)
+    return 0;
+  return gemv_batch_scratch(d_in, d_out, batch);
+}
+
+extern "C" bc_status bc_gemv_batch(const void* W, int d_in, int d_out, const float* x, const int* idx, int k,
+                                   int batch, float* y, int* n_union, void* scratch, size_t scratch_bytes,
+                                   void* stream) {
+  if (!W || !x || !y || !scratch) return fail(BC_EINVAL, "null pointer");
+  if (batch < 1 || batch > kBatchMax) return fail(BC_EINVAL, "batch %d outside [1, %d]", batch, kBatchMax);
+  if (d_in < 1 || d_in > kMaxSelect) return fail(BC_EINVAL, "d_in %d outside [1, %d]", d_in, kMaxSelect);
+  if (d_out < kColTile || d_out % kColTile) return fail(BC_EINVAL, "d_out must be a positive multiple of 256");
+  if (k < 1 || k > d_in || (!idx && k != d_in)) return fail(BC_EINVAL, "k must be in [1, d_in] (= d_in without idx)");
+  if (scratch_bytes < gemv_batch_scratch(d_in, d_out, batch)) return fail(BC_ENOMEM, "scratch too small");
+  BatchGemvArgs a;
+  memset(&a, 0, sizeof a);
+  a.W = static_cast<const __nv_bfloat16*>(W);
+  a.d_in = d_in;
+  a.d_out = d_out;
+  a.k = k;
+  a.B = batch;
+  a.x = x;
+  a.idx = idx;
+  a.y = y;
+  a.S = gemv_batch_splits(d_in, d_out, k, batch, device_sms());
+  gemv_batch_bind(&a, scratch, n_union);
+  BC_CUDA(launch_gemv_batch(a, static_cast<cudaStream_t>(stream), true), "bc_gemv_batch");
+  return BC_OK;
+}
+
 extern "C" bc_status bc_select_topk(const float* v, int n, int k, int* idx, void* stream) {
   if (!v || !idx) return fail(BC_EINVAL, "null pointer");
   if (n < 1 || n > kMaxSelect || k < 1 || k > n) return fail(BC_EINVAL, "need 1 <= k <= n <= 16384");

@@ -95,3 +95,21 @@ extern "C" bc_status bc_byte_account(const bc_config* c, bc_mode mode, float rp_
   out->pages_kept = K;
   return BC_OK;
 }
+
+// Batch crossover (ByteCross README, "Usage: The byte account"): a batch of
+// `batch` sequences reads the union of its kept projection rows once
+// (fraction union_keep of the weights) while every sequence saves its own
+// KV bytes, so the two savings meet at
+//   n = (1 - union_keep) P_l / (batch (1 - rkv) 2 Hkv hd) tokens.
+extern "C" bc_status bc_crossover_batch(const bc_config* c, double union_keep, double rkv, int batch,
+                                        double* n_star) {
+  if (!c || !n_star) return BC_EINVAL;
+  if (c->hidden < 1 || c->intermediate < 1 || c->n_heads < 1 || c->n_kv_heads < 1 || c->head_dim < 1)
+    return BC_EINVAL;
+  if (!(union_keep > 0 && union_keep <= 1) || !(rkv > 0 && rkv < 1) || batch < 1) return BC_EINVAL;
+  const double d = c->hidden, f = c->intermediate;
+  const double hq = (double)c->n_heads * c->head_dim, hkv = (double)c->n_kv_heads * c->head_dim;
+  const double P_l = d * hq + 2 * d * hkv + hq * d + 3 * d * f;
+  *n_star = (1 - union_keep) * P_l / ((double)batch * (1 - rkv) * 2 * hkv);
+  return BC_OK;
+}

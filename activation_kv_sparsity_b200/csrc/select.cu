@@ -61,7 +61,7 @@ struct SelClusterSmem {
 template <typename StateF>
 __device__ void cluster_topk(const uint32_t* s_key, int s0, int ns, int need, StateF state, uint32_t lo,
                              uint32_t hi, int* out, SelClusterSmem& sm, cg::cluster_group& cl) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x;
   for (int b = tid; b < 2 * 256; b += kSelClThreads) (&sm.hist[0][0])[b] = 0;
   block_minmax<kSelClThreads>(lo, hi, sm.rmin, sm.rmax);
   if (tid == 0) {

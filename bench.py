@@ -620,6 +620,8 @@ def run_kernel_only(args, local):
         return {"kernel": "snap", "ms_per_selection": round(ms, 4), "flops": flops,
                 "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
                 "note": "2 layers at 32K, both passes and the page select; mma.sync m16n8k16, bf16 keys, hi/lo-split queries"}
+    if args.only_kernel == "gemv_batch":
+        return run_batch_gemv(args, dev, stream, cfg)
     if args.only_kernel in ("gemv_gateup", "gemv_gateup_dense"):
         d, d_out = cfg["hidden"], 2 * cfg["intermediate"]
         W = (torch.randn(d, d_out, generator=g, device=dev) * 0.02).to(torch.bfloat16)
@@ -661,6 +663,69 @@ def run_kernel_only(args, local):
     return {"kernel": args.only_kernel, "ms_per_launch": round(ms, 5), "algorithmic_bytes": nbytes,
             "gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "peak": peak, "peak_kind": kind,
             "note": "includes the combine kernel" if args.only_kernel == "attention" else ""}
+
+
+def run_batch_gemv(args, dev, stream, cfg):
+    """The gate/up projection of one layer (4096 -> 28672 columns, rp 0.5)
+    for a batch of B = 1, 2, 4, 8 sequences: one batched GEMV over the union
+    of their kept channels against B separate gathered GEMVs.  The
+    selections are the library's own top-k of the synthetic batch
+    activations.  L2 is flushed (a 256 MB write) before every timed launch,
+    so the separate GEMVs cannot reuse each other's rows from L2."""
+    import torch
+    import activation_kv_sparsity_b200 as bc
+    from synth import batch_activations
+    d, d_out = cfg["hidden"], 2 * cfg["intermediate"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    W = (torch.randn(d, d_out, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    k = math.ceil(0.5 * d - 1e-9)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peak, kind = peaks()
+
+    def timed(fn):
+        ev = []
+        for i in range(args.warmup + args.steps):
+            flush.fill_(i & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            if i >= args.warmup:
+                ev.append((e0, e1))
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+    rows = []
+    for B in (1, 2, 4, 8):
+        X = batch_activations(B, d, device=dev).contiguous()
+        idx = torch.empty(B, k, dtype=torch.int32, device=dev)
+        for b in range(B):
+            bc.select_topk(X[b], k, idx[b], stream)
+        y = torch.empty(B, d_out, device=dev)
+        ys = torch.empty(B, d_out, device=dev)
+        nu = torch.zeros(1, dtype=torch.int32, device=dev)
+        scratch = torch.empty(bc.bc_gemv_batch_scratch_bytes(d, d_out, B), dtype=torch.uint8, device=dev)
+        s1 = torch.zeros(bc.bc_gemv_scratch_bytes(d_out), dtype=torch.uint8, device=dev)
+        ms_b = timed(lambda: bc.gemv_batch(W, X, idx, y, scratch, nu, stream))
+
+        def separate():
+            for b in range(B):
+                bc.gemv(W, X[b], idx[b], ys[b], s1, stream)
+        ms_s = timed(separate)
+        u = int(nu.item())
+        nbytes = u * d_out * 2 + B * (k * 4 + d * 4 + d_out * 4)
+        gbs = nbytes / (ms_b * 1e-3) / 1e9
+        keep = u / d
+        rows.append({"batch": B, "union_rows": u, "union_keep": round(keep, 4),
+                     "ms_batched": round(ms_b, 5), "ms_separate": round(ms_s, 5),
+                     "speedup_vs_separate": round(ms_s / ms_b, 3), "algorithmic_bytes": nbytes,
+                     "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+                     "weight_rows_separate_over_union": round(B * k / u, 3),
+                     "crossover_batch_tokens_rkv0.3": round(bc.crossover_batch(cfg, keep, 0.3, B), 1)})
+    return {"kernel": "gemv_batch", "peak": peak, "peak_kind": kind, "rows": rows,
+            "note": "gate/up of one layer, rp 0.5, batch activations with a shared component (union ~92% at 4); "
+                    "L2 flushed before each timed launch; batched = union + GEMV (+ split reduce)"}
 
 
 GEMV_SITES = ["qkv", "o", "gate_up", "down"]
@@ -744,7 +809,7 @@ def main():
                     help="per-site cost of one step in this mode at the first --contexts value")
     ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
                     help="write profiles/traffic.json from an ncu raw CSV of --only-kernel gemv_gateup")
-    ap.add_argument("--only-kernel", choices=("gemv_gateup", "gemv_gateup_dense", "attention", "snap"),
+    ap.add_argument("--only-kernel", choices=("gemv_gateup", "gemv_gateup_dense", "attention", "snap", "gemv_batch"),
                     help="time one kernel alone on a small case (profiler captures)")
     args = ap.parse_args()
     if args.record_traffic:

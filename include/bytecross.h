@@ -274,6 +274,29 @@ BC_API int bc_gemv_noalloc_max_dout(void);
 BC_API bc_status bc_gemv_noalloc(const void* W, int d_in, int d_out, const float* x, const int* idx, int k,
                                  float* y, void* stream);
 
+/* Batched column-gathered GEMV over the union of the sequences' kept
+ * channels, the projection of a batched decode step (README, "Usage: The byte
+ * account": crossover_batch, where a batch reads the union of its kept
+ * projection weights once).  Each sequence keeps its own channels, so
+ *   y[b][j] = sum over c in S_b of x[b][c] * W[c][j],   b in [0, batch)
+ * is what bc_gemv gives for sequence b alone, while the rows of the union
+ * U = S_0 u ... u S_{batch-1} are read once for the whole batch.
+ * W: device bf16 [d_in][d_out] (input-channel-major); x: device f32
+ * [batch][d_in]; idx: device int32 [batch][k], row b the channels S_b
+ * (any order; duplicates and values outside [0, d_in) are ignored), or NULL
+ * for all d_in channels (then k must equal d_in); y: device f32
+ * [batch][d_out], overwritten; n_union: device int32 [1] that receives |U|,
+ * or NULL.  scratch: device buffer of bc_gemv_batch_scratch_bytes(d_in,
+ * d_out, batch) bytes (union list, masked inputs, split partials; no
+ * zeroing needed).  1 <= batch <= 8, 1 <= k <= d_in <= 16384, d_out a
+ * multiple of 256.  stream: cudaStream_t.  Deterministic: the partial sums
+ * of a column are added in a fixed order.  Invalid sizes: BC_EINVAL; small
+ * scratch: BC_ENOMEM; nothing is launched then. */
+BC_API size_t bc_gemv_batch_scratch_bytes(int d_in, int d_out, int batch);
+BC_API bc_status bc_gemv_batch(const void* W, int d_in, int d_out, const float* x, const int* idx, int k,
+                               int batch, float* y, int* n_union, void* scratch, size_t scratch_bytes,
+                               void* stream);
+
 /* Exact top-k selection: writes to idx (device int32 [k]) the k indices of
  * largest |v| (v: device f32 [n]), ascending; ties go to the lower index.
  * 1 <= k <= n <= 16384. */
@@ -329,6 +352,17 @@ typedef struct {
 
 BC_API bc_status bc_byte_account(const bc_config* cfg, bc_mode mode, float rp, float rkv,
                                  long long n_ctx, int sinks, int recent, int page, bc_bytes* out);
+
+/* Batch crossover (README, "Usage: The byte account", crossover_batch): the
+ * context, in tokens, at which the projection branch of a batch of `batch`
+ * sequences -- which reads the union of its sequences' kept weight rows,
+ * a fraction union_keep of them -- saves as many bytes as the KV branch at
+ * keep rkv, which saves per sequence:
+ *   n* = (1 - union_keep) P_l / (batch (1 - rkv) 2 Hkv hd)
+ * (P_l as for bc_byte_account's n_star).  Host only.  BC_EINVAL unless
+ * 0 < union_keep <= 1, 0 < rkv < 1 and batch >= 1. */
+BC_API bc_status bc_crossover_batch(const bc_config* cfg, double union_keep, double rkv, int batch,
+                                    double* n_star);
 
 /* ------------------------------------------------------------------ errors */
 

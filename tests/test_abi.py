@@ -90,6 +90,25 @@ def test_single_kernel_entries_validate_on_host():
     assert bc.bc_attention(p, p, 8, 4, 96, 10, None, 1, 16, p, p, 1 << 20, None) == bc.BC_EINVAL
 
 
+def test_batched_gemv_validates_on_host():
+    p = C.c_void_p(256)
+    big = 1 << 30
+    assert bc.bc_gemv_batch_scratch_bytes(4096, 300, 4) == 0
+    assert bc.bc_gemv_batch_scratch_bytes(4096, 512, 9) == 0
+    assert bc.bc_gemv_batch_scratch_bytes(20000, 512, 2) == 0
+    assert bc.bc_gemv_batch_scratch_bytes(4096, 512, 4) > 4 * 4096 * 4
+    # batch out of range, d_out not a multiple of 256, k > d_in, no idx with
+    # k < d_in, scratch too small: rejected before any launch
+    assert bc.bc_gemv_batch(p, 64, 256, p, p, 8, 0, p, None, p, big, None) == bc.BC_EINVAL
+    assert bc.bc_gemv_batch(p, 64, 256, p, p, 8, 9, p, None, p, big, None) == bc.BC_EINVAL
+    assert bc.bc_gemv_batch(p, 64, 300, p, p, 8, 2, p, None, p, big, None) == bc.BC_EINVAL
+    assert bc.bc_gemv_batch(p, 64, 256, p, p, 65, 2, p, None, p, big, None) == bc.BC_EINVAL
+    assert bc.bc_gemv_batch(p, 64, 256, p, None, 8, 2, p, None, p, big, None) == bc.BC_EINVAL
+    assert bc.bc_gemv_batch(None, 64, 256, p, p, 8, 2, p, None, p, big, None) == bc.BC_EINVAL
+    need = bc.bc_gemv_batch_scratch_bytes(64, 256, 2)
+    assert bc.bc_gemv_batch(p, 64, 256, p, p, 8, 2, p, None, p, need - 1, None) == bc.BC_ENOMEM
+
+
 MODELS = {k: dict(v, page=16) for k, v in GOLD["models"].items()}
 
 
@@ -98,6 +117,26 @@ def test_library_crossover_matches_printed(case):
     got = bc.byte_account(MODELS[case["model"]], "both", 1024, rp=case["rp"], rkv=case["rkv"])
     assert round(got["n_star"] / 1024, case["digits"]) == pytest.approx(case["printed"])
     assert got["n_star"] == pytest.approx(ba.crossover(MODELS[case["model"]], case["rp"], case["rkv"]), rel=1e-6)
+
+
+def test_library_crossover_batch_matches_printed_and_oracle():
+    c = GOLD["crossover_batch_k"][0]
+    m = MODELS[c["model"]]
+    got = bc.crossover_batch(m, c["union_keep"], c["rkv"], c["batch"])
+    assert round(got / 1024, c["digits"]) == pytest.approx(c["printed"])
+    for keep, rkv, batch in [(0.92, 0.3, 4), (0.75, 0.5, 2), (0.996, 0.2, 8), (0.5, 0.3, 1)]:
+        assert got_eq(bc.crossover_batch(m, keep, rkv, batch), ba.crossover_batch(m, keep, rkv, batch))
+    # batch 1 with union_keep = rp is Equation 5's crossover
+    assert got_eq(bc.crossover_batch(m, 0.5, 0.3, 1), ba.crossover(m, 0.5, 0.3))
+    out = C.c_double()
+    cfg = bc.config(m, 1)
+    assert bc.bc_crossover_batch(C.byref(cfg), 0.0, 0.3, 4, C.byref(out)) == bc.BC_EINVAL
+    assert bc.bc_crossover_batch(C.byref(cfg), 0.9, 1.0, 4, C.byref(out)) == bc.BC_EINVAL
+    assert bc.bc_crossover_batch(C.byref(cfg), 0.9, 0.3, 0, C.byref(out)) == bc.BC_EINVAL
+
+
+def got_eq(a, b):
+    return a == pytest.approx(b, rel=1e-12)
 
 
 def test_library_bound_and_ff_match_printed():

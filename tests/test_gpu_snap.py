@@ -80,16 +80,21 @@ def _snap_model(t, n, n_obs=8):
 
 
 def test_snap_steps_match_oracle(tiny):
-    """Ten steps from 6 tokens before a page boundary: the oracle replays the
-    GPU's kept pages (checked exact above) and attends over them plus the
+    """Ten steps from 6 tokens before a page boundary: the oracle makes its
+    own selection from the same observation queries (its scores leave a
+    margin of 0.4% at every cut, far above the scorer's rounding, so the
+    GPU's kept pages must equal it) and attends over those pages plus the
     page the steps open."""
     cfg = tiny["cfg"]
     n = 2048 - 6
     m, k, v = _snap_model(tiny, n)
-    _, kept = _snap_traces(m, cfg)
-    P_snap = -(-n // 16)
+    _, gpu_kept = _snap_traces(m, cfg)
     cache = od.Cache(cfg, n + 64)
     cache.extend(bits(k), bits(v))
+    kept, _, P_snap = od.snap_select(cfg, cache, obs_queries(cfg, 8, seed=12).double().numpy(),
+                                     SEL["rkv"], SEL["sinks"], SEL["recent"])
+    for key, pages in kept.items():
+        assert gpu_kept[key].tolist() == pages.tolist(), key
     logits = torch.empty(cfg["vocab"], device=DEV)
     for i, tok in enumerate(tokens(10, cfg["vocab"], seed=4)):
         m.step(tok, "snap", logits, **SEL)
