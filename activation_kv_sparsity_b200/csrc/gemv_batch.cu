@@ -11,26 +11,25 @@
 // "Usage: The byte account": crossover_batch, where a batch reads the union
 // of its kept projection weights once per step).
 //
-// Two launches, chained by programmatic dependent launch:
+// Three launches, chained by programmatic dependent launch:
 //   k_union         one CTA: marks every listed channel with its sequences'
-//                   bits in shared memory, compacts the marked channels
-//                   (ascending) into the union list, and writes the union
-//                   rows' inputs row-major, B floats per row, 0 where a
-//                   sequence did not keep the row; |U| to device memory.
+//                   bits in shared memory and compacts the marked channels
+//                   (ascending) into the union list, each entry the channel
+//                   with its sequences' bits; |U| to device memory.
 //   k_gemv_batch<B> a column tile of 256 outputs (8 per lane: one 16-byte
 //                   load of a row segment) and a contiguous run of at most
 //                   1024 union rows per CTA, cut from the device-side |U|
 //                   (the grid is planned for the largest union,
 //                   min(d_in, B*k), and to fill whole waves of 2 CTAs per
-//                   SM).  The run's channel ids and inputs are staged in
-//                   shared memory first, so a row's weight load waits on no
-//                   global load; 8 warps, 16 row segments per lane in flight
+//                   SM).  The run's channel ids and inputs (0 where a
+//                   sequence did not keep the row) are gathered into shared
+//                   memory first, so a row's weight load waits on no global
+//                   load; 8 warps, 16 row segments per lane in flight
 //                   (8 for B > 4), B x 8 accumulators per lane; warps reduced
-//                   in shared memory.  A tile split over several runs adds
-//                   one stage through scratch: each run writes its partial
-//                   and takes an atomic ticket; the last to arrive (no
-//                   waiting) sums the runs' partials in run order, so the
-//                   result is deterministic.
+//                   in shared memory; a tile split over several runs writes
+//                   one partial per run.
+//   k_batch_reduce  sums the runs' partials in run order (deterministic);
+//                   skipped when one run covers a tile.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -54,15 +53,24 @@ __global__ void __launch_bounds__(kUnionThreads) k_union(BatchGemvArgs a) {
   for (int c = tid; c < a.d_in; c += kUnionThreads) s_mark[c] = a.idx ? 0u : all;
   __syncthreads();
   if (a.idx) {
+    // four independent list loads per thread in flight, then their marks
     const int total = a.B * a.k;
-    for (int e = tid; e < total; e += kUnionThreads) {
-      const int c = a.idx[e];
-      if (c >= 0 && c < a.d_in) atomicOr(&s_mark[c], 1u << (e / a.k));
+    for (int e0 = tid; e0 < total; e0 += 4 * kUnionThreads) {
+      int c[4];
+      #pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * kUnionThreads;
+        c[u] = e < total ? a.idx[e] : -1;
+      }
+      #pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c[u] >= 0 && c[u] < a.d_in) atomicOr(&s_mark[c[u]], 1u << ((e0 + u * kUnionThreads) / a.k));
     }
     __syncthreads();
   }
   // thread t owns the contiguous channels [t*per, (t+1)*per): the union
-  // comes out ascending
+  // comes out ascending; an entry packs the channel (low 16 bits) with its
+  // sequences' bits (bits 16-23)
   const int per = (a.d_in + kUnionThreads - 1) / kUnionThreads;
   const int c0 = min(a.d_in, tid * per), c1 = min(a.d_in, c0 + per);
   int cnt = 0;
@@ -71,15 +79,9 @@ __global__ void __launch_bounds__(kUnionThreads) k_union(BatchGemvArgs a) {
   int off = block_excl_scan<kUnionThreads>(cnt, s_red, &total);
   for (int c = c0; c < c1; ++c) {
     const uint32_t m = s_mark[c];
-    if (!m) continue;
-    a.ulist[off] = c;
-    for (int b = 0; b < a.B; ++b)
-      a.xu[(size_t)off * a.B + b] = ((m >> b) & 1u) ? a.x[(size_t)b * a.d_in + c] : 0.f;
-    ++off;
+    if (m) a.ulist[off++] = (int)((uint32_t)c | (m << 16));
   }
   if (tid == 0) *a.n_union = total;
-  // the GEMV's tile tickets start at zero on every call
-  for (int t = tid; t < a.d_out / kBatchCols; t += kUnionThreads) a.tickets[t] = 0u;
 }
 
 __device__ __forceinline__ void fma8b(float* acc, float xv, const uint4& w) {
@@ -129,9 +131,15 @@ __global__ void __launch_bounds__(kBatchThreads, 2) k_gemv_batch(BatchGemvArgs a
   const int n = *a.n_union;
   const int r0 = (int)((long long)run * n / a.S), r1 = (int)((long long)(run + 1) * n / a.S);
   const int len = r1 - r0;                      // <= kBatchRunCap: S is planned for it
-  // the run's channel ids and inputs, once per CTA
-  for (int i = tid; i < len; i += kBatchThreads) s_id[i] = a.ulist[r0 + i];
-  for (int i = tid; i < len * B; i += kBatchThreads) s_x[i] = a.xu[(size_t)r0 * B + i];
+  // the run's channel ids and masked inputs, gathered once per CTA
+  #pragma unroll 4
+  for (int i = tid; i < len * B; i += kBatchThreads) {
+    const int row = i / B, b = i - row * B;
+    const uint32_t e = (uint32_t)__ldg(a.ulist + r0 + row);
+    const int c = (int)(e & 0xFFFFu);
+    if (b == 0) s_id[row] = c;
+    s_x[i] = ((e >> (16 + b)) & 1u) ? __ldg(a.x + (size_t)b * a.d_in + c) : 0.f;
+  }
   __syncthreads();
   const __nv_bfloat16* Wc = a.W + (size_t)tile * kBatchCols + lane * 8;
   float acc[B][8];
@@ -156,10 +164,6 @@ __global__ void __launch_bounds__(kBatchThreads, 2) k_gemv_batch(BatchGemvArgs a
       }
     }
   }
-  // warps reduced in shared memory; with one run the sums are the outputs,
-  // otherwise the run's partial goes to scratch and the tile's last CTA to
-  // arrive (atomic ticket, no waiting) adds the runs' partials in run order
-  const size_t col = (size_t)tile * kBatchCols + tid;
   float* out = a.S == 1 ? a.y : a.partial + (size_t)run * B * a.d_out;
   #pragma unroll
   for (int b = 0; b < B; ++b) {
@@ -170,23 +174,31 @@ __global__ void __launch_bounds__(kBatchThreads, 2) k_gemv_batch(BatchGemvArgs a
     float v = 0.f;
     #pragma unroll
     for (int w = 0; w < kBatchWarps; ++w) v += s_red[w][tid];
-    out[(size_t)b * a.d_out + col] = v;
+    out[(size_t)b * a.d_out + (size_t)tile * kBatchCols + tid] = v;
     __syncthreads();
   }
-  if (a.S == 1) return;
-  __shared__ unsigned s_last;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = atomicAdd(&a.tickets[tile], 1u) == (unsigned)(a.S - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  #pragma unroll
-  for (int b = 0; b < B; ++b) {
-    float v = 0.f;
-    for (int q = 0; q < a.S; ++q) v += __ldcg(a.partial + ((size_t)q * B + b) * a.d_out + col);
-    a.y[(size_t)b * a.d_out + col] = v;
+}
+
+__global__ void k_batch_reduce(BatchGemvArgs a) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  const int n = a.B * a.d_out;
+  if (e >= n) return;
+  // four runs' partials in flight at a time, added in run order
+  const float* p = a.partial + e;
+  float v = 0.f;
+  int s = 0;
+  for (; s + 4 <= a.S; s += 4) {
+    const float p0 = p[(size_t)s * n], p1 = p[(size_t)(s + 1) * n];
+    const float p2 = p[(size_t)(s + 2) * n], p3 = p[(size_t)(s + 3) * n];
+    v += p0;
+    v += p1;
+    v += p2;
+    v += p3;
   }
+  for (; s < a.S; ++s) v += p[(size_t)s * n];
+  a.y[e] = v;
 }
 
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -214,20 +226,15 @@ int gemv_batch_splits(int d_in, int d_out, int k, int B, int sms) {
 }
 
 size_t gemv_batch_scratch(int d_in, int d_out, int B) {
-  return al256(4ull * d_in) + al256(4ull * d_in * B) + 256 + al256(4ull * (d_out / kBatchCols)) +
-         al256(4ull * kBatchMaxSplit * B * d_out);
+  return al256(4ull * d_in) + 256 + al256(4ull * kBatchMaxSplit * B * d_out);
 }
 
 void gemv_batch_bind(BatchGemvArgs* a, void* scratch, int* n_union) {
   char* p = static_cast<char*>(scratch);
   a->ulist = reinterpret_cast<int*>(p);
   p += al256(4ull * a->d_in);
-  a->xu = reinterpret_cast<float*>(p);
-  p += al256(4ull * a->d_in * a->B);
   a->n_union = n_union ? n_union : reinterpret_cast<int*>(p);
   p += 256;
-  a->tickets = reinterpret_cast<unsigned*>(p);
-  p += al256(4ull * (a->d_out / kBatchCols));
   a->partial = reinterpret_cast<float*>(p);
 }
 
@@ -274,7 +281,12 @@ cudaError_t launch_gemv_batch(const BatchGemvArgs& a, cudaStream_t st, bool pdl)
     case 7: e = launch_b<7>(cfg, a); break;
     default: e = launch_b<8>(cfg, a); break;
   }
-  return e;
+  if (e != cudaSuccess || a.S == 1) return e;
+  cudaLaunchConfig_t r = cfg;
+  r.gridDim = dim3((a.B * a.d_out + 255) / 256);
+  r.blockDim = dim3(256);
+  r.dynamicSmemBytes = 0;
+  return cudaLaunchKernelEx(&r, k_batch_reduce, a);
 }
 
 }  // namespace bc

@@ -149,17 +149,15 @@ struct BatchGemvArgs {
   int d_in, d_out, k, B;
   const float* x;                 // [B][d_in]
   const int* idx;                 // [B][k] kept channels per sequence, or nullptr for all (k == d_in)
-  int* ulist;                     // [d_in] union U, ascending (first |U| entries)
-  float* xu;                      // [d_in][B] inputs of the union rows, 0 where a sequence did not keep the row
+  int* ulist;                     // [d_in] union U, ascending (first |U| entries): channel | sequence bits << 16
   int* n_union;                   // |U|
-  unsigned* tickets;              // [d_out / 256] arrivals per column tile (zeroed by the union kernel)
   float* partial;                 // [S][B][d_out] (S > 1 only)
   int S;                          // row runs per column tile
   float* y;                       // [B][d_out]
 };
 int gemv_batch_splits(int d_in, int d_out, int k, int B, int sms);
 size_t gemv_batch_scratch(int d_in, int d_out, int B);
-// Carves ulist / xu / n_union / tickets / partial out of scratch (n_union stays in
+// Carves ulist / n_union / partial out of scratch (n_union stays in
 // scratch unless given).
 void gemv_batch_bind(BatchGemvArgs* a, void* scratch, int* n_union);
 cudaError_t launch_gemv_batch(const BatchGemvArgs& a, cudaStream_t st, bool pdl);
