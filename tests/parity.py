@@ -2,6 +2,8 @@
 the same seeded inputs and compare them the way the tests state."""
 from __future__ import annotations
 
+import math
+
 import numpy as np
 import torch
 
@@ -59,18 +61,38 @@ def forced_from(tr, act: bool, kvsel: bool):
     return forced
 
 
+def topk_of(score, k):
+    """The k largest entries of score, ties to the lower index, ascending."""
+    order = np.lexsort((np.arange(score.size), -score))
+    return np.sort(order[:k])
+
+
+def pages_of(score, rkv, sinks, recent):
+    """Forced pages (the first `sinks`, the last `recent`) plus the best
+    scored others up to K = clamp(ceil(rkv*P - 1e-9), |F|, P), ascending."""
+    P = score.size
+    forced = sorted(set(range(min(sinks, P))) | set(range(max(P - recent, 0), P)))
+    K = max(len(forced), min(P, math.ceil(rkv * P - 1e-9)))
+    fset = set(forced)
+    free = np.array([p for p in range(P) if p not in fset], dtype=np.int64)
+    chosen = free[np.lexsort((free, -score[free]))[:K - len(forced)]] if K > len(forced) else []
+    return np.sort(np.concatenate([np.asarray(forced, dtype=np.int64), np.asarray(chosen, dtype=np.int64)]))
+
+
 def check_selection_exact(tr, rp, rkv, sinks, recent, act, kvsel):
-    """The oracle's selection routines, fed the GPU's own pre-selection scores
-    (fp32 values, compared exactly in fp64), must return the GPU's sets."""
+    """Every GPU set is exactly the selection its own pre-selection scores
+    define (a property of the GPU's output checked here, in the test, on the
+    GPU's own fp32 values; the oracle never sees them)."""
     for l, r in enumerate(tr):
         if act:
             for site, _, _ in SITES:
-                score = {"qkv": r["xn"], "o": r["attn"], "gu": r["xn2"], "d": r["h"]}[site]
-                np.testing.assert_array_equal(od.channel_select(score, rp), r["s_" + site],
+                score = np.abs({"qkv": r["xn"], "o": r["attn"], "gu": r["xn2"], "d": r["h"]}[site])
+                k = max(1, min(score.size, math.ceil(rp * score.size - 1e-9)))
+                np.testing.assert_array_equal(topk_of(score, k), r["s_" + site],
                                               err_msg=f"layer {l} site {site}")
         if kvsel:
             for h in range(r["pages"].shape[0]):
-                np.testing.assert_array_equal(od.page_select(r["page_scores"][h], rkv, sinks, recent),
+                np.testing.assert_array_equal(pages_of(r["page_scores"][h], rkv, sinks, recent),
                                               r["pages"][h], err_msg=f"layer {l} kv head {h}")
 
 
@@ -87,9 +109,13 @@ def check_selection_near(own, gpu_set, cut_from_scores, k):
     return diff.size
 
 
-def compare_step(cfg, w_bits, cache, token, mode, rp, rkv, sinks, recent, logits_gpu, tr):
-    """Runs the oracle on the GPU's selections and compares; returns the
-    oracle's logits and trace."""
+def compare_step(cfg, w_bits, cache, token, mode, rp, rkv, sinks, recent, logits_gpu, tr, layers=None):
+    """Checks the GPU's sets (exact on its own scores), then runs the oracle
+    over the whole step from its own inputs, told only the GPU's index sets
+    (integers: where fp32 and fp64 scores straddle a cut, both choices are
+    correct), and compares every set with the oracle's own choice (near-ties
+    only), the hidden states of `layers` (default all) and the logits.
+    Returns the oracle's logits and trace."""
     act = mode in ("act", "both")
     kvsel = mode in ("kv", "both")
     check_selection_exact(tr, rp, rkv, sinks, recent, act, kvsel)
@@ -97,8 +123,9 @@ def compare_step(cfg, w_bits, cache, token, mode, rp, rkv, sinks, recent, logits
     ref = od.decode_step(cfg, w_bits, cache, token, mode, rp=rp, rkv=rkv, sinks=sinks, recent=recent,
                          forced=forced_from(tr, act, kvsel), trace=trace)
     for l, r in enumerate(tr):
-        e = max_rel(r["x"], trace[l]["x"])
-        assert e < REL_TOL, f"layer {l} hidden rel err {e}"
+        if layers is None or l in layers:
+            e = max_rel(r["x"], trace[l]["x"])
+            assert e < REL_TOL, f"layer {l} hidden rel err {e}"
         if act:
             for site, _, _ in SITES:
                 own_scores = np.abs({"qkv": trace[l]["xn"], "o": trace[l]["attn"], "gu": trace[l]["xn2"],
