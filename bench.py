@@ -378,7 +378,7 @@ def run_ours(args, rank, ws, local):
         "crossings": {"byte_account": crossings, "measured": cross_measured},
     }
     if rank == 0 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(args, w, model, head_ctx)
+        result["cpu_baseline"] = cpu_baseline(args, w, head_ctx)
     del attn
     model.close()
     return result
@@ -477,13 +477,13 @@ def oracle_sample(w_host, cache, n_ctx, mode, layer, lm_rows, token=7):
     return t1 - t0, t2 - t1
 
 
-def host_sample_inputs(w_dev, model, n_ctx, n_layers):
+def host_sample_inputs(w_dev, n_ctx, n_layers):
     """Host copies of what the oracle sample needs: the first n_layers'
-    weights, the LM head slice, and those layers' KV read back from the pool."""
-    import numpy as np
-    import torch
+    weights, the LM head slice, and a KV cache of those layers drawn from the
+    input generator (the same recipe and seed as the timed cache; the oracle
+    never reads the library's pool)."""
     from oracle import decoder as od
-    from synth import LLAMA_8B, bf16_bits
+    from synth import LLAMA_8B, bf16_bits, kv_chunks
     cfg = LLAMA_8B
     wh = {}
     for name in ("attn_norm", "mlp_norm", "wqkv_t", "wo_t", "wgu_t", "wd_t"):
@@ -491,18 +491,11 @@ def host_sample_inputs(w_dev, model, n_ctx, n_layers):
     wh["embed"] = bf16_bits(w_dev["embed"][:16])
     wh["final_norm"] = bf16_bits(w_dev["final_norm"])
     wh["lm_head"] = bf16_bits(w_dev["lm_head"][: cfg["vocab"] // 32])
-    Pmax = model.c.max_ctx // 16 + (model.c.max_ctx % 16 > 0)
-    pool = model.kv_pool.view(torch.bfloat16).view(cfg["n_layers"], cfg["n_kv_heads"], Pmax, 2, 16,
-                                                   cfg["head_dim"])
-    P = -(-n_ctx // 16)
-    cache = od.Cache(dict(cfg, n_layers=n_layers), n_ctx + 1)
-    for l in range(n_layers):
-        kp = pool[l, :, :P, 0].reshape(cfg["n_kv_heads"], P * 16, -1)[:, :n_ctx]
-        vp = pool[l, :, :P, 1].reshape(cfg["n_kv_heads"], P * 16, -1)[:, :n_ctx]
-        cache.k[l, :, :n_ctx] = bf16_bits(kp)
-        cache.v[l, :, :n_ctx] = bf16_bits(vp)
+    small = dict(cfg, n_layers=n_layers)
+    cache = od.Cache(small, n_ctx + 1)
+    for k, v in kv_chunks(small, n_ctx, seed=1, device=w_dev["embed"].device):
+        cache.extend(bf16_bits(k), bf16_bits(v))
     cache.n = n_ctx
-    del np
     return wh, cache
 
 
@@ -514,13 +507,13 @@ def cpu_threads():
         return os.cpu_count()
 
 
-def cpu_baseline(args, w_dev, model, n_ctx):
+def cpu_baseline(args, w_dev, n_ctx):
     """The oracle as it stands, on the host cores: layers 0-3 of one decode
     step of the headline cell plus 1/32 of the LM head, scaled to a full step."""
     from synth import LLAMA_8B
     cfg = LLAMA_8B
     nl = 4
-    wh, cache = host_sample_inputs(w_dev, model, n_ctx, nl)
+    wh, cache = host_sample_inputs(w_dev, n_ctx, nl)
     layer_s, head_s = [], 0.0
     for l in range(nl):
         a, b = oracle_sample(wh, cache, n_ctx, HEAD_MODE, l, cfg["vocab"] // 32)
