@@ -287,9 +287,9 @@ BC_API bc_status bc_gemv_noalloc(const void* W, int d_in, int d_out, const float
  * for all d_in channels (then k must equal d_in); y: device f32
  * [batch][d_out], overwritten; n_union: device int32 [1] that receives |U|,
  * or NULL.  scratch: device buffer of bc_gemv_batch_scratch_bytes(d_in,
- * d_out, batch) bytes (union list, masked inputs, split partials; no
- * zeroing needed).  1 <= batch <= 8, 1 <= k <= d_in <= 16384, d_out a
- * multiple of 256.  stream: cudaStream_t.  Deterministic: the partial sums
+ * d_out, batch) bytes (union list and split partials; no zeroing
+ * needed).  1 <= batch <= 8, 1 <= k <= d_in <= 16384, d_out a multiple of
+ * 256.  stream: cudaStream_t.  Deterministic: the partial sums
  * of a column are added in a fixed order.  Invalid sizes: BC_EINVAL; small
  * scratch: BC_ENOMEM; nothing is launched then. */
 BC_API size_t bc_gemv_batch_scratch_bytes(int d_in, int d_out, int batch);
