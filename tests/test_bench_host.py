@@ -1,0 +1,82 @@
+"""Host-side logic of the benchmark, on CPU: the measured crossing's linear
+interpolation, the cost-aware fit (it must recover a bandwidth and per-mode
+fixed costs it was built from, and predict the crossing of that model), the
+byte-account crossing by bisection, and the per-site labels of a traced
+step."""
+import pytest
+
+import activation_kv_sparsity_b200 as bc
+import bench
+from synth import LLAMA_8B
+
+CTX = (2048, 8192, 32768, 65536, 131072)
+
+
+def test_measured_crossing_interpolates_linearly():
+    cells = {}
+    for n, (a, k) in zip(CTX, [(3.0, 3.7), (3.2, 4.0), (3.6, 4.1), (4.3, 4.4), (5.5, 5.0)]):
+        cells[("act", n)] = {"ms_per_step": a}
+        cells[("kv", n)] = {"ms_per_step": k}
+    got = bench.measured_crossing(cells, CTX)["act_vs_kv_tokens"]
+    # act - kv: -0.1 at 64K, +0.5 at 128K -> 65536 + 65536 * 0.1 / 0.6
+    assert got == pytest.approx(65536 + 65536 * 0.1 / 0.6, abs=0.1)
+
+
+def test_measured_crossing_absent():
+    cells = {(m, n): {"ms_per_step": 1.0 if m == "act" else 2.0} for m in ("act", "kv") for n in CTX}
+    assert bench.measured_crossing(cells, CTX)["act_vs_kv_tokens"] is None
+    assert bench.measured_crossing({}, CTX) == {"act_vs_kv_tokens": None}
+
+
+def _model_cells(bw_gbs, cost_ms):
+    cells = {}
+    for m in ("dense", "act", "kv"):
+        for n in CTX:
+            b = bc.byte_account(LLAMA_8B, m, n, **{k: v for k, v in bench.KEEP.items()
+                                                  if m != "dense" or k in ("sinks", "recent")})["impl_total_bytes"]
+            cells[(m, n)] = {"bytes_per_step": b, "ms_per_step": b / (bw_gbs * 1e9) * 1e3 + cost_ms[m]}
+    return cells
+
+
+def test_cost_aware_fit_recovers_its_model():
+    costs = {"dense": 1.3, "act": 1.9, "kv": 1.6}
+    cells = _model_cells(6700.0, costs)
+    fit = bench.cost_aware_prediction(cells, CTX, LLAMA_8B, bc)
+    assert fit["fit_gbs"] == pytest.approx(6700.0, rel=1e-6)
+    for m, c in costs.items():
+        assert fit["fixed_cost_ms"][m] == pytest.approx(c, abs=1e-3)
+    n = fit["predicted_act_vs_kv_tokens"]
+
+    def t(mode, ctx):
+        kw = dict(bench.KEEP)
+        return bc.byte_account(LLAMA_8B, mode, ctx, **kw)["impl_total_bytes"] / 6700e9 * 1e3 + costs[mode]
+    assert t("act", n - 1) < t("kv", n - 1) and t("act", n) >= t("kv", n)
+
+
+def test_cost_aware_fit_needs_all_modes():
+    cells = _model_cells(6700.0, {"dense": 1.0, "act": 1.0, "kv": 1.0})
+    del cells[("kv", 2048)]
+    assert bench.cost_aware_prediction(cells, CTX, LLAMA_8B, bc) is None
+
+
+def test_impl_crossing_is_where_the_byte_counts_meet():
+    n = bench.impl_crossing(bc, LLAMA_8B, 0.5, 0.3)
+
+    def diff(ctx):
+        a = bc.byte_account(LLAMA_8B, "act", ctx, rp=0.5)["impl_total_bytes"]
+        k = bc.byte_account(LLAMA_8B, "kv", ctx, rkv=0.3)["impl_total_bytes"]
+        return a - k
+    assert diff(n - 1) < 0 <= diff(n)
+    # the paper form's n* (Equation 5) is below it: the page bounds cost the KV branch bytes
+    assert bc.byte_account(LLAMA_8B, "both", 0, rp=0.5, rkv=0.3)["n_star"] < n
+
+
+def test_site_labels_follow_the_projection_order():
+    names = ["k_select_cta", "k_gemv", "k_pages", "k_page_select_cta", "k_attn", "k_select_cta", "k_gemv",
+             "k_select_cta", "k_gemv", "k_select", "k_gemv", "k_lmhead"]
+    sites, gemvs = [], 0
+    for nm in names:
+        sites.append(bench.site_of(nm, gemvs))
+        gemvs += "k_gemv" in nm
+    assert sites == ["sel_qkv", "qkv", "page_scores", "page_select", "attn", "sel_o", "o", "sel_gate_up",
+                     "gate_up", "sel_down", "down", "k_lmhead"]
