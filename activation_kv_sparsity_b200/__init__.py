@@ -19,8 +19,8 @@ _lib = C.CDLL(LIB_PATH)
 
 # ------------------------------------------------------------------ enums
 BC_OK, BC_EINVAL, BC_ENOMEM, BC_ECAPACITY, BC_ECUDA, BC_ETIMEOUT = range(6)
-BC_DENSE, BC_ACT, BC_KV, BC_BOTH, BC_SNAP = range(5)
-MODES = {"dense": BC_DENSE, "act": BC_ACT, "kv": BC_KV, "both": BC_BOTH, "snap": BC_SNAP}
+BC_DENSE, BC_ACT, BC_KV, BC_BOTH, BC_SNAP, BC_MASKED = range(6)
+MODES = {"dense": BC_DENSE, "act": BC_ACT, "kv": BC_KV, "both": BC_BOTH, "snap": BC_SNAP, "masked": BC_MASKED}
 (BC_TRACE_XN, BC_TRACE_SEL_QKV, BC_TRACE_Q, BC_TRACE_ATTN, BC_TRACE_SEL_O, BC_TRACE_XN2,
  BC_TRACE_SEL_GU, BC_TRACE_H, BC_TRACE_SEL_D, BC_TRACE_X, BC_TRACE_PAGE_SCORES, BC_TRACE_PAGES,
  BC_TRACE_QKV, BC_TRACE_SNAP_SCORES, BC_TRACE_SNAP_PAGES) = range(15)
@@ -59,9 +59,9 @@ _SIGS = {
     "bc_launch_count": (C.c_longlong, [_P]),
     "bc_kv_reset": (C.c_int, [_P, C.c_int]),
     "bc_kv_append": (C.c_int, [_P, _P, _P, C.c_int]),
-    "bc_kv_snap_select": (C.c_int, [_P, _P, C.c_int, C.c_float, C.c_int, C.c_int]),
-    "bc_decode_step": (C.c_int, [_P, C.c_int, C.c_int, C.c_float, C.c_float, C.c_int, C.c_int, C.c_int, _P]),
-    "bc_decode_step_host": (C.c_int, [_P, C.c_int, C.c_int, C.c_float, C.c_float, C.c_int, C.c_int, C.c_int, _P]),
+    "bc_kv_snap_select": (C.c_int, [_P, _P, C.c_int, C.c_double, C.c_int, C.c_int]),
+    "bc_decode_step": (C.c_int, [_P, C.c_int, C.c_int, C.c_double, C.c_double, C.c_int, C.c_int, C.c_int, _P]),
+    "bc_decode_step_host": (C.c_int, [_P, C.c_int, C.c_int, C.c_double, C.c_double, C.c_int, C.c_int, C.c_int, _P]),
     "bc_trace": (C.c_int, [_P, C.c_int, C.c_int, C.POINTER(_P), C.POINTER(C.c_int), C.POINTER(C.c_int)]),
     "bc_gemv_scratch_bytes": (C.c_size_t, [C.c_int]),
     "bc_gemv": (C.c_int, [_P, C.c_int, C.c_int, _P, _P, C.c_int, _P, _P, C.c_size_t, _P]),
@@ -73,7 +73,7 @@ _SIGS = {
     "bc_attention_scratch_bytes": (C.c_size_t, [C.c_int, C.c_int]),
     "bc_attention": (C.c_int, [_P, _P, C.c_int, C.c_int, C.c_int, C.c_int, _P, C.c_int, C.c_int, _P, _P,
                                C.c_size_t, _P]),
-    "bc_byte_account": (C.c_int, [C.POINTER(bc_config), C.c_int, C.c_float, C.c_float, C.c_longlong, C.c_int,
+    "bc_byte_account": (C.c_int, [C.POINTER(bc_config), C.c_int, C.c_double, C.c_double, C.c_longlong, C.c_int,
                                   C.c_int, C.c_int, C.POINTER(bc_bytes)]),
     "bc_crossover_batch": (C.c_int, [C.POINTER(bc_config), C.c_double, C.c_double, C.c_int,
                                      C.POINTER(C.c_double)]),

@@ -198,7 +198,7 @@ struct NodeRec {
 struct StepGraph {
   bc_mode mode;
   int psel;              // page-select variant of the captured page counts (kv modes)
-  float rp, rkv;
+  double rp, rkv;
   int sinks, recent;
   cudaGraph_t graph;
   cudaGraphExec_t exec;
@@ -299,7 +299,7 @@ extern "C" bc_status bc_kv_reset(bc_model* m, int n_ctx) {
   return BC_OK;
 }
 
-extern "C" bc_status bc_kv_snap_select(bc_model* m, const float* q_obs, int n_obs, float rkv, int sinks,
+extern "C" bc_status bc_kv_snap_select(bc_model* m, const float* q_obs, int n_obs, double rkv, int sinks,
                                        int recent) {
   if (!m || !q_obs) return fail(BC_EINVAL, "null argument");
   const bc_config& c = m->cfg;
@@ -307,13 +307,13 @@ extern "C" bc_status bc_kv_snap_select(bc_model* m, const float* q_obs, int n_ob
   const int G = c.n_heads / c.n_kv_heads, Hkv = c.n_kv_heads, L = c.n_layers;
   if (n_obs < 1 || n_obs * G > kSnapMaxQ)
     return fail(BC_EINVAL, "n_obs %d outside [1, %d]", n_obs, kSnapMaxQ / G);
-  if (!(rkv > 0.f && rkv <= 1.f)) return fail(BC_EINVAL, "rkv %g outside (0, 1]", rkv);
+  if (!(rkv > 0.0 && rkv <= 1.0)) return fail(BC_EINVAL, "rkv %g outside (0, 1]", rkv);
   if (sinks < 0 || recent < 1) return fail(BC_EINVAL, "sinks must be >= 0 and recent >= 1");
   if (m->n < 1) return fail(BC_EINVAL, "the cache holds no tokens");
   const int n = m->n, P = (n + kPage - 1) / kPage, Pmax = y.Pmax;
   const int sink_end = std::min(sinks, P), rec_begin = std::max(P - recent, 0);
   const int n_forced = sink_end + (P - std::max(rec_begin, sink_end));
-  const int K = std::max(n_forced, (int)std::min<double>(P, ceil((double)rkv * P - 1e-9)));
+  const int K = std::max(n_forced, (int)std::min<double>(P, ceil(rkv * P - 1e-9)));
   const size_t kv_layer = (size_t)Hkv * Pmax * 2 * kPage * c.head_dim;
   m->snap_valid = false;
   for (int l = 0; l < L; ++l) {
@@ -366,20 +366,20 @@ extern "C" bc_status bc_kv_append(bc_model* m, const void* k, const void* v, int
   return BC_OK;
 }
 
-static int keep_count(float ratio, int n) {
-  const double v = ceil((double)ratio * n - 1e-9);
+static int keep_count(double ratio, int n) {
+  const double v = ceil(ratio * n - 1e-9);
   return (int)std::max(1.0, std::min((double)n, v));
 }
 
-static bc_status check_step(const bc_model* m, bc_mode mode, float rp, float rkv, int sinks,
+static bc_status check_step(const bc_model* m, bc_mode mode, double rp, double rkv, int sinks,
                             int recent, int page) {
   if (!m) return fail(BC_EINVAL, "null model");
-  if (mode < BC_DENSE || mode > BC_SNAP) return fail(BC_EINVAL, "bad mode %d", (int)mode);
+  if (mode < BC_DENSE || mode > BC_MASKED) return fail(BC_EINVAL, "bad mode %d", (int)mode);
   if (mode == BC_SNAP && !m->snap_valid)
     return fail(BC_EINVAL, "snap mode needs a selection (bc_kv_snap_select) since the last append or reset");
   if (page != m->cfg.page) return fail(BC_EINVAL, "page %d differs from the model's %d", page, m->cfg.page);
-  if (!(rp > 0.f && rp <= 1.f)) return fail(BC_EINVAL, "rp %g outside (0, 1]", rp);
-  if (!(rkv > 0.f && rkv <= 1.f)) return fail(BC_EINVAL, "rkv %g outside (0, 1]", rkv);
+  if (!(rp > 0.0 && rp <= 1.0)) return fail(BC_EINVAL, "rp %g outside (0, 1]", rp);
+  if (!(rkv > 0.0 && rkv <= 1.0)) return fail(BC_EINVAL, "rkv %g outside (0, 1]", rkv);
   if (sinks < 0 || recent < 1) return fail(BC_EINVAL, "sinks must be >= 0 and recent >= 1");
   if (m->n + 1 > m->cfg.max_ctx) return fail(BC_ECAPACITY, "KV cache full (%d tokens)", m->n);
   return BC_OK;
@@ -462,10 +462,11 @@ static bool record(std::vector<NodeRec>* rec, cudaStream_t st, int kind, int lay
 struct StepShape {
   int pos, n_tok, P, K, splits, pps;
   int list_len, tail0;      // attention page list: listed entries, then pages tail0, tail0+1, ...
+  int mask_on, mask_sink_end, mask_rec_begin;   // BC_MASKED: the window's pages unmasked
   int k_qkv, k_o, k_gu, k_d;
 };
 
-static StepShape step_shape(const bc_model* m, bc_mode mode, float rp, float rkv, int sinks, int recent) {
+static StepShape step_shape(const bc_model* m, bc_mode mode, double rp, double rkv, int sinks, int recent) {
   const bc_config& c = m->cfg;
   const bool act = mode == BC_ACT || mode == BC_BOTH;
   const bool kvs = mode == BC_KV || mode == BC_BOTH;
@@ -476,6 +477,9 @@ static StepShape step_shape(const bc_model* m, bc_mode mode, float rp, float rkv
   sh.K = sh.P;
   sh.list_len = 0;
   sh.tail0 = 0;
+  sh.mask_on = mode == BC_MASKED;
+  sh.mask_sink_end = std::min(sinks, sh.P);
+  sh.mask_rec_begin = std::max(sh.P - recent, 0);
   if (mode == BC_SNAP) {
     sh.K = m->snap_K + std::max(0, sh.P - m->snap_P);
     sh.list_len = m->snap_K;
@@ -484,7 +488,7 @@ static StepShape step_shape(const bc_model* m, bc_mode mode, float rp, float rkv
   if (kvs) {
     const int sink_end = std::min(sinks, sh.P), rec_begin = std::max(sh.P - recent, 0);
     const int n_forced = sink_end + (sh.P - std::max(rec_begin, sink_end));
-    const int want = (int)std::min<double>(sh.P, ceil((double)rkv * sh.P - 1e-9));
+    const int want = (int)std::min<double>(sh.P, ceil(rkv * sh.P - 1e-9));
     sh.K = std::max(n_forced, want);
     sh.list_len = sh.K;
   }
@@ -512,7 +516,7 @@ static void commit_step(bc_model* m, bc_mode mode, const StepShape& sh, long lon
 
 // Enqueues one decode step on m->stream (launching, or recording into a
 // capture when rec is given).  Returns the number of kernels in *launches.
-static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, float rkv, int sinks,
+static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, double rp, double rkv, int sinks,
                               int recent, float* logits, std::vector<NodeRec>* rec, long long* n_launch) {
   const bc_config& c = m->cfg;
   const Layout& y = m->lay;
@@ -605,6 +609,7 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
       launches += 2;
     }
     AttnArgs aa;
+    memset(&aa, 0, sizeof aa);
     aa.q = q;
     aa.kv = kvl;
     aa.pages = kvs ? pages : mode == BC_SNAP ? at<int>(m, y.snap_pages) + (size_t)l * Hkv * Pmax : nullptr;
@@ -618,6 +623,9 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
     aa.n_tok = n_tok;
     aa.splits = splits;
     aa.pages_per_split = pps;
+    aa.mask_on = sh.mask_on;
+    aa.mask_sink_end = sh.mask_sink_end;
+    aa.mask_rec_begin = sh.mask_rec_begin;
     aa.part_o = at<float>(m, y.part_o);
     aa.part_ml = at<float>(m, y.part_ml);
     aa.counters = att_counters;
@@ -664,7 +672,7 @@ static bc_status enqueue_step(bc_model* m, int token, bc_mode mode, float rp, fl
 }
 
 // Captures the step for this configuration on the private stream.
-static bc_status capture_step(bc_model* m, int token, bc_mode mode, float rp, float rkv, int sinks,
+static bc_status capture_step(bc_model* m, int token, bc_mode mode, double rp, double rkv, int sinks,
                               int recent, float* logits, StepGraph** out) {
   if (!m->cap_stream) BC_CUDA(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking), "capture stream");
   StepGraph* g = new StepGraph();
@@ -732,6 +740,8 @@ static cudaError_t launch_step_graph(bc_model* m, StepGraph* g, int token, const
         r.args.a.n_tok = sh.n_tok;
         r.args.a.splits = sh.splits;
         r.args.a.pages_per_split = sh.pps;
+        r.args.a.mask_sink_end = sh.mask_sink_end;
+        r.args.a.mask_rec_begin = sh.mask_rec_begin;
         kp.gridDim = dim3(sh.splits, c.n_kv_heads);
         break;
       case NK_LMHEAD:
@@ -746,7 +756,7 @@ static cudaError_t launch_step_graph(bc_model* m, StepGraph* g, int token, const
   return cudaGraphLaunch(g->exec, m->stream);
 }
 
-static bc_status run_step(bc_model* m, int token, bc_mode mode, float rp, float rkv, int sinks, int recent,
+static bc_status run_step(bc_model* m, int token, bc_mode mode, double rp, double rkv, int sinks, int recent,
                           float* logits) {
   const StepShape sh = step_shape(m, mode, rp, rkv, sinks, recent);
   if (m->use_graphs) {
@@ -788,7 +798,7 @@ static bc_status run_step(bc_model* m, int token, bc_mode mode, float rp, float 
   return s;
 }
 
-extern "C" bc_status bc_decode_step(bc_model* m, int token, bc_mode mode, float rp, float rkv,
+extern "C" bc_status bc_decode_step(bc_model* m, int token, bc_mode mode, double rp, double rkv,
                                     int sinks, int recent, int page, float* logits) {
   bc_status s = check_step(m, mode, rp, rkv, sinks, recent, page);
   if (s != BC_OK) return s;
@@ -797,7 +807,7 @@ extern "C" bc_status bc_decode_step(bc_model* m, int token, bc_mode mode, float 
   return run_step(m, token, mode, rp, rkv, sinks, recent, logits);
 }
 
-extern "C" bc_status bc_decode_step_host(bc_model* m, int token, bc_mode mode, float rp, float rkv,
+extern "C" bc_status bc_decode_step_host(bc_model* m, int token, bc_mode mode, double rp, double rkv,
                                          int sinks, int recent, int page, float* logits_host) {
   bc_status s = check_step(m, mode, rp, rkv, sinks, recent, page);
   if (s != BC_OK) return s;
@@ -945,6 +955,7 @@ extern "C" bc_status bc_attention(const float* q, const void* kv, int n_kv_heads
   const int nq = n_kv_heads * group;
   if (scratch_bytes < bc_attention_scratch_bytes(nq, head_dim)) return fail(BC_ENOMEM, "scratch too small");
   AttnArgs a;
+  memset(&a, 0, sizeof a);
   a.q = q;
   a.kv = static_cast<const __nv_bfloat16*>(kv);
   a.pages = pages;

@@ -24,6 +24,12 @@
 // the pages tail0, tail0 + 1, ... (the pages begun after a once-after-prefill
 // selection).
 //
+// With mask_on the kernel is the masked dense baseline of the README's FAQ
+// ("A KV method reports a speedup above its byte bound"): it reads every
+// page of the list and adds an additive mask, 0 on the window's pages (the
+// sinks and the recent pages) and -inf elsewhere, to the logits.  Masked
+// pages cost their bytes and contribute nothing.
+//
 // Partials (m, l, o) per (query head, split) use base-2 logits.  The last
 // CTA of each kv head to finish (an atomic ticket, no spinning) merges them:
 // o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, summing in split order.
@@ -118,7 +124,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn(AttnArgs a) {
     }
   };
   auto process_page = [&](int page, uint4* k0, uint4* k1, uint4* v0, uint4* v1) {
-    const int valid = min(kPage, a.n_tok - page * kPage);
+    const bool masked = a.mask_on && page >= a.mask_sink_end && page < a.mask_rec_begin;
+    const int valid = masked ? 0 : min(kPage, a.n_tok - page * kPage);
     if (g >= valid) {
       #pragma unroll
       for (int u = 0; u < U4; ++u) v0[u] = make_uint4(0, 0, 0, 0);
@@ -148,10 +155,12 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn(AttnArgs a) {
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     const float m_new = fmaxf(m_run, mx);
-    const float alpha = exp2f(m_run - m_new);
+    // no valid logit yet (only masked pages so far): scale by 2^0, not 2^(-inf + inf)
+    const float m_use = m_new == -INFINITY ? 0.f : m_new;
+    const float alpha = exp2f(m_run - m_use);
     float p[4];
     #pragma unroll
-    for (int j = 0; j < 4; ++j) p[j] = exp2f(sc[j] - m_new);
+    for (int j = 0; j < 4; ++j) p[j] = exp2f(sc[j] - m_use);
     l_run = l_run * alpha + (p[0] + p[1]) + (p[2] + p[3]);
     m_run = m_new;
     #pragma unroll

@@ -26,14 +26,13 @@ static long long keep_rows(double ratio, long long n) {
   return std::max(1LL, std::min(n, (long long)v));
 }
 
-extern "C" bc_status bc_byte_account(const bc_config* c, bc_mode mode, float rp_f, float rkv_f,
+extern "C" bc_status bc_byte_account(const bc_config* c, bc_mode mode, double rp, double rkv,
                                      long long n_ctx, int sinks, int recent, int page, bc_bytes* out) {
   if (!c || !out) return BC_EINVAL;
   if (c->n_layers < 1 || c->hidden < 1 || c->intermediate < 1 || c->n_heads < 1 || c->n_kv_heads < 1 ||
       c->head_dim < 1 || c->vocab < 1 || page < 1 || n_ctx < 0 || sinks < 0 || recent < 1)
     return BC_EINVAL;
-  if (mode < BC_DENSE || mode > BC_SNAP) return BC_EINVAL;
-  const double rp = rp_f, rkv = rkv_f;
+  if (mode < BC_DENSE || mode > BC_MASKED) return BC_EINVAL;
   if (!(rp > 0 && rp <= 1) || !(rkv > 0 && rkv <= 1)) return BC_EINVAL;
   const bool act = mode == BC_ACT || mode == BC_BOTH;
   const bool kvs = mode == BC_KV || mode == BC_BOTH;

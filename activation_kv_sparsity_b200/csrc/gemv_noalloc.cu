@@ -10,7 +10,7 @@
 // entry point keeps the scratch in a file-scope __device__ array instead, so
 // the caller passes only W, x, the channel list and y.
 //
-// The array holds kNoAllocMaxDout * 256 bytes + the tickets (8 MiB + 512 B)
+// The array holds kNoAllocMaxDout * 256 bytes + the tickets (8 MiB + 1 KiB)
 // and lives on every GPU that loads the library until the process exits.
 // Its device address is looked up once per device, on the first call made
 // while that device is current; make that first call before capturing a

@@ -112,6 +112,10 @@ struct AttnArgs {
   int Hkv, G, hd, Pmax, n_pages, n_tok;
   int list_len, tail0;            // entries >= list_len are pages tail0, tail0+1, ... (not listed)
   int splits, pages_per_split;
+  // additive page mask (the masked dense baseline): with mask_on, a page p
+  // of the list adds 0 to its logits when p < mask_sink_end or
+  // p >= mask_rec_begin and -inf otherwise; its bytes are read either way
+  int mask_on, mask_sink_end, mask_rec_begin;
   float* part_o;                  // [Hkv*G][kMaxSplits][hd]
   float* part_ml;                 // [Hkv*G][kMaxSplits][2]
   unsigned* counters;             // [Hkv], zero between launches

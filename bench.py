@@ -41,17 +41,38 @@ METRIC = "decode tok/s per mode (dense/act/KV/both), 2K–128K ctx; HBM GB/s vs 
 HEAD_MODE, HEAD_CTX = "both", 32768
 KEEP = dict(rp=0.5, rkv=0.3, sinks=1, recent=16)
 CONTEXTS = (131072, 65536, 32768, 8192, 2048)         # descending: every cell sees pristine synthetic KV
-MODE_KW = {"dense": dict(), "act": dict(rp=0.5), "kv": dict(rkv=0.3, sinks=1, recent=16),
-           "both": dict(rp=0.5, rkv=0.3, sinks=1, recent=16),
-           # the pages' KV window baseline: the kv mode with no scored pages
-           # (K = |F|: the sink page and the 16 recent pages)
-           "window": dict(rkv=1e-6, sinks=1, recent=16),
-           # the pages' own KV mode: one selection after prefill (16 observation
-           # positions per query head), then steps over the frozen pages
-           "snap": dict(rkv=0.3, sinks=1, recent=16)}
+FORCED = dict(sinks=1, recent=16)                     # 1 sink page, 16 recent pages = 256 tokens
+# Bench cells: name -> (library mode, keep arguments).  The keep pairs are the
+# ones the ByteCross README times (rp 0.7 / 0.5, rkv 0.3 / 0.5).
+CELLS = {
+    "dense": ("dense", {}),
+    "act": ("act", dict(rp=0.5)),
+    "kv": ("kv", dict(rkv=0.3, **FORCED)),
+    "both": ("both", dict(rp=0.5, rkv=0.3, **FORCED)),
+    # the pages' KV window baseline: the kv mode with no scored pages
+    # (K = |F|: the sink page and the 16 recent pages)
+    "window": ("kv", dict(rkv=1e-6, **FORCED)),
+    # the same window computed by the masked dense baseline: every KV byte
+    # read, an additive mask keeping the window's pages
+    "masked": ("masked", dict(FORCED)),
+    # the pages' own KV mode: one selection after prefill (16 observation
+    # positions per query head), then steps over the frozen pages
+    "snap": ("snap", dict(rkv=0.3, **FORCED)),
+    "act@0.7": ("act", dict(rp=0.7)),
+    "kv@0.5": ("kv", dict(rkv=0.5, **FORCED)),
+    "both@0.7/0.3": ("both", dict(rp=0.7, rkv=0.3, **FORCED)),
+    "both@0.5/0.5": ("both", dict(rp=0.5, rkv=0.5, **FORCED)),
+}
+DEFAULT_CELLS = ["dense", "act", "kv", "both", "window", "masked", "snap", "act@0.7", "kv@0.5",
+                 "both@0.7/0.3", "both@0.5/0.5"]
+MODE_KW = {name: kw for name, (_, kw) in CELLS.items()}
 SNAP_OBS = 16
-LIB_MODE = {"window": "kv"}                          # bench cells that run a library mode
-CROSS_PAIRS = ((0.7, 0.3), (0.5, 0.3), (0.5, 0.5))
+# the keep pairs whose act-vs-kv crossings are located: (rp, rkv) -> (act cell, kv cell)
+CROSS_CELLS = {(0.7, 0.3): ("act@0.7", "kv"), (0.5, 0.3): ("act", "kv"), (0.5, 0.5): ("act", "kv@0.5")}
+# the crossing sweep: 2K, then 4K to 128K in 4K steps, each context timed in
+# every sweep cell back to back (a block), blocks repeated
+SWEEP_CONTEXTS = tuple([2048] + [4096 * i for i in range(1, 33)])
+SWEEP_CELLS = ("dense", "act@0.7", "act", "kv", "kv@0.5")
 
 
 def peaks():
@@ -193,6 +214,14 @@ def traffic_record(kernel):
 
 # ------------------------------------------------------------------ our arm
 
+def cell_kw(name):
+    """Full keep arguments of a cell (ratios default to 1, the forced pages
+    to the benchmark's 1 sink page and 16 recent pages)."""
+    kw = dict(rp=1.0, rkv=1.0, **FORCED)
+    kw.update(CELLS[name][1])
+    return kw
+
+
 def run_ours(args, rank, ws, local):
     import torch
     import activation_kv_sparsity_b200 as bc
@@ -202,11 +231,13 @@ def run_ours(args, rank, ws, local):
     torch.cuda.set_device(dev)
     cfg = LLAMA_8B
     contexts = sorted(set(args.contexts), reverse=True)
+    sweep_ctx = sorted((n for n in SWEEP_CONTEXTS if n <= max(contexts)), reverse=True) if args.sweep_blocks else []
     steps, warm = args.steps, args.warmup
-    max_ctx = max(contexts) + warm + steps + 32
+    sw_steps = min(steps, args.sweep_steps)
+    max_ctx = max(contexts + sweep_ctx) + warm + steps + 32
     w = make_weights(cfg, seed=0, device=dev)
     model = bc.Model(cfg, w, max_ctx)
-    for k, v in kv_chunks(cfg, max(contexts), seed=1, device=dev):
+    for k, v in kv_chunks(cfg, max(contexts + sweep_ctx), seed=1, device=dev):
         model.append(k, v)
     torch.cuda.synchronize()
     stream = model.stream
@@ -218,12 +249,12 @@ def run_ours(args, rank, ws, local):
 
     q_obs = obs_queries(cfg, SNAP_OBS, device=dev) if "snap" in args.modes else None
     snap_select_ms = {}
+    host_enqueue = {}
 
-    def time_cell(mode, n):
-        kw = MODE_KW[mode]
-        lib = LIB_MODE.get(mode, mode)
+    def time_cell(name, n, k_steps):
+        lib, kw = CELLS[name]
         model.reset(n)
-        if mode == "snap":
+        if lib == "snap":
             # the selection is paid once per prefill: timed apart from the steps
             s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s0.record(stream)
@@ -240,15 +271,28 @@ def run_ours(args, rank, ws, local):
         t0 = time.time()
         e0.record(stream)
         h0 = time.perf_counter()
-        for i in range(steps):
+        for i in range(k_steps):
             model.step(toks[warm + i], lib, logits, **kw)
-        host_enqueue[(mode, n)] = (time.perf_counter() - h0) * 1e3 / steps
+        host_enqueue[(name, n)] = (time.perf_counter() - h0) * 1e3 / k_steps
         e1.record(stream)
         torch.cuda.synchronize()
         clocks.window(t0, time.time())
         barrier(ws)
-        ms = max_over_ranks(e0.elapsed_time(e1) / steps, ws, dev)
+        ms = max_over_ranks(e0.elapsed_time(e1) / k_steps, ws, dev)
         return ms, model.launches() - l0
+
+    def step_bytes(name, n, k_steps):
+        """Byte account of the timed steps (contexts n+warm .. n+warm+k_steps-1), averaged."""
+        lib, _ = CELLS[name]
+        kw = cell_kw(name)
+        if lib == "snap":
+            # the step right after the selection at n, plus every token
+            # appended since (each is read: frozen partial page, new pages)
+            base = bc.byte_account(cfg, "snap", n, **kw)
+            tok_bytes = cfg["n_layers"] * cfg["n_kv_heads"] * 2 * cfg["head_dim"] * 2
+            return base, base["impl_total_bytes"] + tok_bytes * (warm + (k_steps - 1) / 2.0)
+        accs = [bc.byte_account(cfg, lib, n + warm + i, **kw) for i in range(k_steps)]
+        return accs[0], sum(a["impl_total_bytes"] for a in accs) / k_steps
 
     def time_e2e(n):
         # end to end through the public host-buffer entry point, at context n
@@ -269,39 +313,44 @@ def run_ours(args, rank, ws, local):
 
     e2e = None
     cells = {}
-    host_enqueue = {}
     for n in contexts:
         if n == HEAD_CTX or (e2e is None and n == min(contexts)):
             e2e = time_e2e(n)
-        for mode in args.modes:
-            ms, launches = time_cell(mode, n)
-            kw = dict(KEEP)
-            kw.update(MODE_KW[mode])
-            # the timed steps run at contexts n+warm .. n+warm+steps-1: average their byte accounts
-            accs = [bc.byte_account(cfg, LIB_MODE.get(mode, mode), n + warm + i, **kw) for i in range(steps)]
-            acc = dict(accs[0])
-            acc["impl_total_bytes"] = sum(a["impl_total_bytes"] for a in accs) / steps
-            if mode == "snap":
-                # the step right after the selection at n, plus every token
-                # appended since (each is read: frozen partial page, new pages)
-                base = bc.byte_account(cfg, "snap", n, **kw)["impl_total_bytes"]
-                tok_bytes = cfg["n_layers"] * cfg["n_kv_heads"] * 2 * cfg["head_dim"] * 2
-                acc["impl_total_bytes"] = base + tok_bytes * (warm + (steps - 1) / 2.0)
-            gbs = acc["impl_total_bytes"] / (ms * 1e-3) / 1e9
-            cells[(mode, n)] = dict(mode=mode, context=n, ms_per_step=round(ms, 4),
-                                    tok_s=round(1000.0 / ms, 2), bytes_per_step=acc["impl_total_bytes"],
+        for name in args.modes:
+            ms, launches = time_cell(name, n, steps)
+            acc, nbytes = step_bytes(name, n, steps)
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            cells[(name, n)] = dict(mode=name, context=n, ms_per_step=round(ms, 4),
+                                    tok_s=round(1000.0 / ms, 2), bytes_per_step=nbytes,
                                     gbs=round(gbs, 1), frac_of_measured_peak=round(gbs / peak, 4),
                                     paper_bound=round(acc["bound"], 4), launches_per_step=launches // steps,
-                                    host_enqueue_ms=round(host_enqueue[(mode, n)], 4))
-            if mode == "snap":
-                cells[(mode, n)]["selection_ms_once"] = round(snap_select_ms[n], 3)
+                                    host_enqueue_ms=round(host_enqueue[(name, n)], 4))
+            if CELLS[name][0] == "snap":
+                cells[(name, n)]["selection_ms_once"] = round(snap_select_ms[n], 3)
     for n in contexts:
         if ("dense", n) not in cells:
             continue
-        d = cells[("dense", n)]["ms_per_step"]
-        for mode in ("act", "kv", "both", "window", "snap"):
-            if (mode, n) in cells:
-                cells[(mode, n)]["speedup_vs_dense"] = round(d / cells[(mode, n)]["ms_per_step"], 4)
+        d = cells[("dense", n)]
+        for name in args.modes:
+            c = cells.get((name, n))
+            if c is None or name == "dense":
+                continue
+            c["speedup_vs_dense"] = round(d["ms_per_step"] / c["ms_per_step"], 4)
+            # the bound a pure byte count allows: dense bytes over this cell's bytes
+            c["byte_bound_vs_dense"] = round(d["bytes_per_step"] / c["bytes_per_step"], 4)
+        if ("window", n) in cells and ("masked", n) in cells:
+            cells[("window", n)]["speedup_vs_masked_dense"] = round(
+                cells[("masked", n)]["ms_per_step"] / cells[("window", n)]["ms_per_step"], 4)
+
+    # the crossing sweep: blocks of every sweep cell at every context
+    sweep = []
+    for b in range(args.sweep_blocks):
+        block = {}
+        for n in sweep_ctx:
+            for name in SWEEP_CELLS:
+                ms, _ = time_cell(name, n, sw_steps)
+                block[(name, n)] = {"ms_per_step": ms, "bytes_per_step": step_bytes(name, n, sw_steps)[1]}
+        sweep.append(block)
 
     head = cells.get((HEAD_MODE, HEAD_CTX)) or cells.get((HEAD_MODE, contexts[0])) or next(iter(cells.values()))
     head_ctx = head["context"]
@@ -332,22 +381,7 @@ def run_ours(args, rank, ws, local):
     gemv_bytes = kq * d_out * 2 + kq * 8            # weight rows + index/activation reads
     achieved = gemv_bytes / (gemv_ms * 1e-3) / 1e9
 
-    # attention at the headline context: dense page list of one layer
-    # (second kernel of interest), timed through the single-kernel entry
-    # point over 8 layers' pages
-    attn = None
-
     clk = clocks.summary()
-    # measured crossing against the byte account: the paper form (Equation 5)
-    # and this implementation's bytes (which add the page bounds the scorer reads)
-    crossings = {}
-    for rp, rkv in CROSS_PAIRS:
-        acc = bc.byte_account(cfg, "both", 1024, rp=rp, rkv=rkv)
-        crossings[f"{rp}/{rkv}"] = {"n_star_tokens": round(acc["n_star"], 1),
-                                    "n_star_impl_tokens": impl_crossing(bc, cfg, rp, rkv)}
-    cross_measured = measured_crossing(cells, contexts)
-    cross_measured["cost_aware_prediction"] = cost_aware_prediction(cells, contexts, cfg, bc)
-
     result = {
         "metric": METRIC,
         "value": round(replica_throughput(steps, head["ms_per_step"] * steps / 1000.0, ws, dev), 2),
@@ -375,13 +409,60 @@ def run_ours(args, rank, ws, local):
         "clocks": clk,
         "e2e": e2e,
         "modes": [cells[k] for k in sorted(cells, key=lambda k: (k[1], k[0]))],
-        "crossings": {"byte_account": crossings, "measured": cross_measured},
+        "crossings": crossing_report(bc, cfg, cells, contexts, sweep, sweep_ctx, sw_steps),
     }
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args, w, head_ctx)
-    del attn
     model.close()
     return result
+
+
+def crossing_report(bc, cfg, cells, contexts, sweep, sweep_ctx, sw_steps):
+    """Per keep pair: the paper-form n* (Equation 5), this implementation's
+    byte crossing, the crossings measured in every sweep block, and the
+    cost-aware prediction fitted on the sweep with its error."""
+    out = {"sweep": {"contexts": sorted(sweep_ctx), "cells": list(SWEEP_CELLS), "blocks": len(sweep),
+                     "steps_per_cell": sw_steps,
+                     "note": "each block times every sweep cell at every context back to back (contexts "
+                             "descending); a crossing is where t(act) - t(kv) turns non-negative, linearly "
+                             "interpolated between neighbouring contexts"}}
+    fit = None
+    if sweep:
+        asc = sorted(sweep_ctx)
+        mean_cells = {(c, n): {"ms_per_step": statistics.mean(b[(c, n)]["ms_per_step"] for b in sweep),
+                               "bytes_per_step": sweep[0][(c, n)]["bytes_per_step"]}
+                      for c in SWEEP_CELLS for n in asc}
+        fit = cost_aware_fit(mean_cells, asc, SWEEP_CELLS)
+        out["sweep"]["ms_mean"] = {c: [round(mean_cells[(c, n)]["ms_per_step"], 4) for n in asc]
+                                   for c in SWEEP_CELLS}
+        if fit:
+            out["cost_aware_fit"] = {"fit_gbs": round(1.0 / fit[0], 1),
+                                     "fixed_cost_ms": {c: round(v * 1e3, 4) for c, v in fit[1].items()}}
+    pairs = {}
+    for (rp, rkv), (ca, ck) in CROSS_CELLS.items():
+        acc = bc.byte_account(cfg, "both", 1024, rp=rp, rkv=rkv)
+        row = {"act_cell": ca, "kv_cell": ck, "n_star_tokens": round(acc["n_star"], 1),
+               "n_star_impl_tokens": impl_crossing(bc, cfg, rp, rkv)}
+        if sweep:
+            asc = sorted(sweep_ctx)
+            per_block = [crossing_of([(n, b[(ca, n)]["ms_per_step"] - b[(ck, n)]["ms_per_step"]) for n in asc])
+                         for b in sweep]
+            row["measured_tokens_per_block"] = per_block
+            found = [x for x in per_block if x is not None]
+            row["measured_tokens"] = round(statistics.mean(found), 1) if found else None
+            if found:
+                row["measured_range_tokens"] = [min(found), max(found)]
+            if fit:
+                pred = predicted_crossing(bc, cfg, fit[0], fit[1], ca, ck)
+                row["cost_aware_predicted_tokens"] = pred
+                if pred is not None and found:
+                    row["prediction_error_tokens"] = round(pred - row["measured_tokens"], 1)
+        pairs[f"{rp}/{rkv}"] = row
+    out["pairs"] = pairs
+    # the coarse cells of the main sweep, for reference (the headline keep pair)
+    out["coarse_act_vs_kv"] = measured_crossing(cells, contexts)
+    out["coarse_act_vs_kv"]["cost_aware_prediction"] = cost_aware_prediction(cells, contexts, cfg, bc)
+    return out
 
 
 def impl_crossing(bc, cfg, rp, rkv, sinks=1, recent=16):
@@ -403,57 +484,75 @@ def impl_crossing(bc, cfg, rp, rkv, sinks=1, recent=16):
     return hi
 
 
-def cost_aware_prediction(cells, contexts, cfg, bc):
-    """The pages' cost-aware prediction restated for this library: per mode,
-    step time = byte-account bytes / B + c (one bandwidth B for all modes,
-    one fixed per-step kernel cost c per mode), fitted by least squares over
-    the sampled contexts; the predicted crossing is where the act and kv fits
-    meet.  Returns the fit and the predicted crossing in tokens."""
+def cost_aware_fit(cells, contexts, kinds):
+    """The pages' cost-aware model restated for this library: per cell kind,
+    step time = byte-account bytes / B + c (one bandwidth B for all kinds,
+    one fixed per-step kernel cost c per kind), fitted by least squares over
+    the sampled contexts.  Returns (1/B in s per GB, {kind: c in s}) or None
+    when a cell is missing."""
     import numpy as np
-    modes = [m for m in ("dense", "act", "kv") if all((m, n) in cells for n in contexts)]
-    if len(modes) < 3:
+    kinds = list(kinds)
+    if not all((m, n) in cells for m in kinds for n in contexts):
         return None
     rows, ys = [], []
-    for j, m in enumerate(modes):
+    for j, m in enumerate(kinds):
         for n in contexts:
             c = cells[(m, n)]
-            r = [c["bytes_per_step"] / 1e9] + [1.0 if k == j else 0.0 for k in range(len(modes))]
-            rows.append(r)
+            rows.append([c["bytes_per_step"] / 1e9] + [1.0 if k == j else 0.0 for k in range(len(kinds))])
             ys.append(c["ms_per_step"] * 1e-3)
     sol, *_ = np.linalg.lstsq(np.array(rows), np.array(ys), rcond=None)
-    inv_bw, costs = sol[0], dict(zip(modes, sol[1:]))
-    kw = dict(KEEP)
+    return sol[0], dict(zip(kinds, sol[1:]))
 
-    def t(mode, n):
-        return bc.byte_account(cfg, mode, n, **kw)["impl_total_bytes"] / 1e9 * inv_bw + costs[mode]
+
+def predicted_crossing(bc, cfg, inv_bw, costs, act_cell, kv_cell):
+    """Context (tokens) at which the fitted act and kv step times meet, by bisection."""
+    def t(cell, n):
+        return bc.byte_account(cfg, CELLS[cell][0], n, **cell_kw(cell))["impl_total_bytes"] / 1e9 * inv_bw \
+            + costs[cell]
     lo, hi = 1, 1 << 21
-    if (t("act", lo) - t("kv", lo)) * (t("act", hi) - t("kv", hi)) > 0:
-        pred = None
-    else:
-        while hi - lo > 1:
-            mid = (lo + hi) // 2
-            if t("act", mid) < t("kv", mid):
-                lo = mid
-            else:
-                hi = mid
-        pred = hi
+    if (t(act_cell, lo) - t(kv_cell, lo)) * (t(act_cell, hi) - t(kv_cell, hi)) > 0:
+        return None
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        if t(act_cell, mid) < t(kv_cell, mid):
+            lo = mid
+        else:
+            hi = mid
+    return hi
+
+
+def cost_aware_prediction(cells, contexts, cfg, bc):
+    """The cost-aware fit over the dense, act and kv cells of the main
+    contexts and its predicted act-vs-kv crossing (rp 0.5, rkv 0.3)."""
+    fit = cost_aware_fit(cells, contexts, ("dense", "act", "kv"))
+    if fit is None:
+        return None
+    inv_bw, costs = fit
     return {"fit_gbs": round(1.0 / inv_bw, 1),
             "fixed_cost_ms": {m: round(v * 1e3, 4) for m, v in costs.items()},
-            "predicted_act_vs_kv_tokens": pred}
+            "predicted_act_vs_kv_tokens": predicted_crossing(bc, cfg, inv_bw, costs, "act", "kv")}
 
 
-def measured_crossing(cells, contexts):
-    """Context where the KV branch starts to beat the projection branch,
-    interpolated linearly between the sampled contexts (the README's
-    convention for latency crossings)."""
-    ctx = sorted(contexts)
-    if not all(("act", n) in cells and ("kv", n) in cells for n in ctx):
-        return {"act_vs_kv_tokens": None}
-    diff = [(n, cells[("act", n)]["ms_per_step"] - cells[("kv", n)]["ms_per_step"]) for n in ctx]
+def crossing_of(diff):
+    """First context where diff = t(act) - t(kv) turns from negative to
+    non-negative, linearly interpolated (the README's convention for latency
+    crossings); diff is [(context, ms)] ascending.  None if it never does."""
     for (n0, d0), (n1, d1) in zip(diff, diff[1:]):
         if d0 < 0 <= d1:
-            return {"act_vs_kv_tokens": round(n0 + (n1 - n0) * (-d0) / (d1 - d0), 1),
-                    "keep": "rp 0.5 (act) vs rkv 0.3 (kv)"}
+            return round(n0 + (n1 - n0) * (-d0) / (d1 - d0), 1)
+    return None
+
+
+def measured_crossing(cells, contexts, act="act", kv="kv"):
+    """Context where the KV branch starts to beat the projection branch over
+    the sampled contexts."""
+    ctx = sorted(contexts)
+    if not all((act, n) in cells and (kv, n) in cells for n in ctx):
+        return {"act_vs_kv_tokens": None}
+    diff = [(n, cells[(act, n)]["ms_per_step"] - cells[(kv, n)]["ms_per_step"]) for n in ctx]
+    got = crossing_of(diff)
+    if got is not None:
+        return {"act_vs_kv_tokens": got, "keep": f"{act} vs {kv}"}
     return {"act_vs_kv_tokens": None, "diff_ms": diff}
 
 
@@ -522,27 +621,28 @@ def cpu_baseline(args, w_dev, n_ctx):
     step_s = statistics.mean(layer_s) * cfg["n_layers"] + head_s * 32
     return {"value": round(1.0 / step_s, 5), "unit": "tok/s", "cores": cpu_threads(), "kind": "oracle",
             "sample": f"fp64 oracle, {HEAD_MODE} mode at {n_ctx} context: layers 0-{nl - 1} of one step "
-                      f"(mean {statistics.mean(layer_s):.2f} s/layer) x {cfg['n_layers']} layers + 1/32 of the "
-                      f"LM head x 32 ({head_s * 32:.2f} s)",
-            "seconds_per_step": round(step_s, 2)}
+                      f"(mean {statistics.mean(layer_s):.2f} s/layer) and 1/32 of the LM head, timed; the value "
+                      f"extrapolates them to {cfg['n_layers']} layers + the whole head ({head_s * 32:.2f} s)",
+            "seconds_timed": round(sum(layer_s) + head_s * nl, 2),
+            "seconds_per_step_extrapolated": round(step_s, 2)}
 
 
 def run_reference(args, rank, ws, local):
-    """The oracle arm: each step is a bounded sample (one layer of the
-    headline cell's step, rotating over layers 0-3, plus 1/32 of the LM head),
-    scaled to a full step."""
+    """The oracle arm.  Each timed step is a bounded sample of the headline
+    cell's decode step: one decoder layer (layers 0-3 in turn) and 1/32 of
+    the LM head, i.e. 1/32 of a step's work; ``value`` counts a sample as
+    1/32 of a token, and ``ms_per_step`` is the time of one sample as timed,
+    so that ``steps * ms_per_step`` is the timed region."""
     import torch
     from synth import LLAMA_8B, kv_chunks, make_weights
     cfg = LLAMA_8B
     nl = 4
     n_ctx = HEAD_CTX
+    frac = 1.0 / cfg["n_layers"]          # a sample's share of a step (one layer; 1/32 of the head)
     # inputs: drawn with the same generators; on the host when no GPU
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
     small = dict(cfg, n_layers=nl)
     w = make_weights(small, seed=0, device=dev)
-
-    class _Pool:          # the oracle reads token-major KV, filled from the draw
-        pass
     from oracle import decoder as od
     from synth import bf16_bits
     cache = od.Cache(small, n_ctx + 1)
@@ -550,24 +650,29 @@ def run_reference(args, rank, ws, local):
         cache.extend(bf16_bits(k), bf16_bits(v))
     wh = {name: bf16_bits(t) for name, t in w.items() if name not in ("embed", "lm_head")}
     wh["embed"] = bf16_bits(w["embed"][:16])
-    wh["lm_head"] = bf16_bits(w["lm_head"][: cfg["vocab"] // 32])
+    wh["lm_head"] = bf16_bits(w["lm_head"][: cfg["vocab"] // cfg["n_layers"]])
     del w
     times = []
     for i in range(args.warmup + args.steps):
-        a, b = oracle_sample(wh, cache, n_ctx, HEAD_MODE, i % nl, cfg["vocab"] // 32)
+        a, b = oracle_sample(wh, cache, n_ctx, HEAD_MODE, i % nl, cfg["vocab"] // cfg["n_layers"])
         if i >= args.warmup:
-            times.append(a * cfg["n_layers"] + b * 32)
-    step_s = statistics.mean(times)
-    val = round(1.0 / step_s, 5)
+            times.append(a + b)
+    sample_s = statistics.mean(times)
+    val = round(frac / sample_s, 6)
+    sample = (f"fp64 oracle, {HEAD_MODE} mode at {n_ctx} context; one timed step = one decoder layer "
+              f"(layers 0-{nl - 1} in turn) + 1/{cfg['n_layers']} of the LM head = 1/{cfg['n_layers']} of a "
+              f"decode step, counted as 1/{cfg['n_layers']} token")
     return {
         "impl": "reference", "metric": METRIC, "value": val, "unit": "tok/s", "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(step_s * 1000, 1), "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": round(sample_s * 1000, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"Llama-3.1-8B-shaped decode, 1 sequence, {n_ctx // 1024}K context, mode {HEAD_MODE} "
                                f"(rp 0.5, rkv 0.3, page 16, 1 sink page, 256 recent tokens)",
                    "global_batch": 1, "seq_len": n_ctx, "parallelism": "host cores"},
-        "cpu_baseline": {"value": val, "unit": "tok/s", "cores": cpu_threads(), "kind": "oracle",
-                         "sample": "per step: one layer of the step (layers 0-3 in turn) x 32 + 1/32 of the LM head x 32"},
+        "tokens_per_timed_step": frac,
+        "timed_seconds": round(sum(times), 2),
+        "full_step_ms_extrapolated": round(sample_s / frac * 1000, 1),
+        "cpu_baseline": {"value": val, "unit": "tok/s", "cores": cpu_threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": val, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -796,8 +901,11 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--contexts", type=int, nargs="+", default=list(CONTEXTS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--modes", nargs="+", default=["dense", "act", "kv", "both", "window", "snap"],
-                    choices=["dense", "act", "kv", "both", "window", "snap"])
+    ap.add_argument("--modes", nargs="+", default=list(DEFAULT_CELLS), choices=list(CELLS),
+                    help="bench cells timed at every --contexts value")
+    ap.add_argument("--sweep-blocks", type=int, default=2,
+                    help="blocks of the 2K-128K crossing sweep in 4K steps (0: no sweep)")
+    ap.add_argument("--sweep-steps", type=int, default=8, help="timed steps per sweep cell (at most --steps)")
     ap.add_argument("--timeline", choices=("dense", "act", "kv", "both"),
                     help="per-site cost of one step in this mode at the first --contexts value")
     ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",

@@ -9,6 +9,10 @@
  * its cache through the same split-K attention kernel (README, "Overview":
  * "One attention kernel for every mode").
  *
+ * Keep ratios are passed as double and every keep count is
+ * ceil(ratio * n - 1e-9) evaluated in double.  (A float ratio would not do:
+ * 0.3f is 0.300000012, which keeps 385 instead of 384 of 1280 pages.)
+ *
  * Conventions shared by every entry point
  *  - Ownership: the caller owns every device buffer (weights, KV pool,
  *    metadata pool, workspace, outputs) and the CUDA stream.  The library owns
@@ -44,8 +48,10 @@ typedef enum {
 } bc_status;
 
 /* Decode modes (ByteCross README, "Timing and quality on a GPU": dense,
- * proj, sel, both). */
-typedef enum { BC_DENSE = 0, BC_ACT = 1, BC_KV = 2, BC_BOTH = 3, BC_SNAP = 4 } bc_mode;
+ * proj, sel, both; BC_SNAP is the once-after-prefill selection; BC_MASKED is
+ * the masked dense baseline of the README's FAQ, "A KV method reports a
+ * speedup above its byte bound"). */
+typedef enum { BC_DENSE = 0, BC_ACT = 1, BC_KV = 2, BC_BOTH = 3, BC_SNAP = 4, BC_MASKED = 5 } bc_mode;
 
 /* Model dimensions: the Hugging Face config fields the README's byte account
  * reads ("Quick start"), plus KV capacity and page size.
@@ -165,7 +171,7 @@ BC_API bc_status bc_kv_append(bc_model* m, const void* k, const void* v, int n_t
  * step graphs); the selection is voided by bc_kv_append and bc_kv_reset.
  * Traces: BC_TRACE_SNAP_SCORES, BC_TRACE_SNAP_PAGES.
  * Errors: BC_EINVAL (no tokens, bad sizes or ratios), BC_ECUDA. */
-BC_API bc_status bc_kv_snap_select(bc_model* m, const float* q_obs, int n_obs, float rkv, int sinks,
+BC_API bc_status bc_kv_snap_select(bc_model* m, const float* q_obs, int n_obs, double rkv, int sinks,
                                    int recent);
 
 /* One decode step at position n = bc_kv_length(m) for input token `token`:
@@ -179,7 +185,12 @@ BC_API bc_status bc_kv_snap_select(bc_model* m, const float* q_obs, int n_obs, f
  *   mode    BC_DENSE, BC_ACT, BC_KV, BC_BOTH, or BC_SNAP: dense projections and
  *           attention over the pages a bc_kv_snap_select kept plus every
  *           page begun since (BC_EINVAL without a valid selection; rp, rkv,
- *           sinks and recent are then not used)
+ *           sinks and recent are then not used), or BC_MASKED: dense
+ *           projections and the KV window (the first `sinks` and the last
+ *           `recent` pages) computed the way the README's masked dense
+ *           baseline does it: attention over every cached page with an
+ *           additive mask (0 on the window's pages, -inf elsewhere), which
+ *           reads every KV byte (rp and rkv are not used)
  *   rp      projection keep ratio in (0,1]; per projection input of width
  *           d_in the k = ceil(rp*d_in - 1e-9) channels of largest |x| are
  *           read (ties: lower index).  Ignored unless mode is ACT or BOTH.
@@ -195,14 +206,14 @@ BC_API bc_status bc_kv_snap_select(bc_model* m, const float* q_obs, int n_obs, f
  *   logits  device f32 [vocab], written.
  * Async on the model's stream; the KV length becomes n + 1.
  * Errors: BC_EINVAL, BC_ECAPACITY (n + 1 > max_ctx), BC_ECUDA. */
-BC_API bc_status bc_decode_step(bc_model* m, int token, bc_mode mode, float rp, float rkv,
+BC_API bc_status bc_decode_step(bc_model* m, int token, bc_mode mode, double rp, double rkv,
                                 int sinks, int recent, int page, float* logits);
 
 /* The same step for callers holding host memory: logits_host is a host
  * f32 [vocab] buffer (pinned memory is fastest).  Enqueues the step, copies
  * the logits device -> host and waits for the stream.  Uses the workspace's
  * logits slot as the device-side destination. */
-BC_API bc_status bc_decode_step_host(bc_model* m, int token, bc_mode mode, float rp, float rkv,
+BC_API bc_status bc_decode_step_host(bc_model* m, int token, bc_mode mode, double rp, double rkv,
                                      int sinks, int recent, int page, float* logits_host);
 
 /* ------------------------------------------------------------------ traces */
@@ -263,7 +274,7 @@ BC_API bc_status bc_gemv(const void* W, int d_in, int d_out, const float* x, con
  * memory and hands the operator only its inputs and outputs, or a serving
  * path that must not call cudaMalloc (it can synchronise the device).
  * The split-K scratch lives in a file-scope __device__ array of
- * 8 MiB + 512 B, held on every GPU that loads the library until exit; d_out
+ * 8 MiB + 1 KiB, held on every GPU that loads the library until exit; d_out
  * above bc_gemv_noalloc_max_dout() (32768) is rejected with BC_EINVAL.  The
  * first call on a device, with that device current, looks the array's
  * address up; make it before any stream capture.  Every call clears the
@@ -327,7 +338,8 @@ BC_API bc_status bc_attention(const float* q, const void* kv, int n_kv_heads, in
  * appended) must move in `mode`.  For BC_SNAP: the step right after a
  * once-after-prefill selection made at n_ctx with rkv, sinks and recent
  * (its kept pages plus a page the token opens; no bounds read); its paper
- * form is the KV branch's. */
+ * form is the KV branch's.  BC_MASKED reads what a dense step reads (every
+ * KV byte; the mask saves none), and its paper form saves nothing. */
 typedef struct {
   /* paper form */
   double weight_bytes;        /* W = 2 L P_l, the seven projections */
@@ -350,7 +362,7 @@ typedef struct {
   long long pages_kept;       /* K per (layer, kv head) */
 } bc_bytes;
 
-BC_API bc_status bc_byte_account(const bc_config* cfg, bc_mode mode, float rp, float rkv,
+BC_API bc_status bc_byte_account(const bc_config* cfg, bc_mode mode, double rp, double rkv,
                                  long long n_ctx, int sinks, int recent, int page, bc_bytes* out);
 
 /* Batch crossover (README, "Usage: The byte account", crossover_batch): the

@@ -140,9 +140,10 @@ def implementation_bytes(cfg, mode, n, rp=1.0, rkv=1.0, sinks=1, recent=16):
     """Bytes one decode step moves at context n (n tokens cached; the step
     appends token n and attends over n+1), enumerated explicitly.
 
-    mode: 'dense', 'act', 'kv', 'both' or 'snap' (the pages a once-after-
+    mode: 'dense', 'act', 'kv', 'both', 'snap' (the pages a once-after-
     prefill selection made at context n kept, plus a page the step's token
-    opens; no bounds are read).  Returns a dict of byte counts.
+    opens; no bounds are read) or 'masked' (the masked dense baseline: every
+    KV byte is read, as in dense).  Returns a dict of byte counts.
     """
     act = mode in ("act", "both")
     kv = mode in ("kv", "both")

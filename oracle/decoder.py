@@ -41,7 +41,13 @@ Readings of what the pages leave open (each is a choice, stated once):
   the kv head's group; the same page rule as above keeps the sinks, the
   recent pages and the best scored others; the kept pages are frozen, and
   every decode step afterwards attends over them plus every page begun
-  after the selection ("snap" mode, dense projections).
+  after the selection ("snap" mode, dense projections);
+* masked dense baseline (README FAQ, "A KV method reports a speedup above
+  its byte bound": a dense attention that masks the cache down to a KV
+  method's pages): dense projections and softmax attention over all n + 1
+  tokens with an additive mask, 0 on the tokens of the window's pages (the
+  first ``sinks`` and the last ``recent`` pages) and -inf on every other
+  token ("masked" mode).  Mathematically it is the KV window.
 
 Arithmetic: fp64 throughout, on bf16 weights and KV widened exactly.
 """
@@ -183,12 +189,15 @@ def snap_select(cfg, cache: "Cache", q_obs, rkv: float, sinks: int, recent: int)
     return kept, scores, -(-n // page)
 
 
-def attention(q: np.ndarray, keys: np.ndarray, values: np.ndarray, tok: np.ndarray):
+def attention(q: np.ndarray, keys: np.ndarray, values: np.ndarray, tok: np.ndarray, bias=None):
     """Softmax attention of the G query heads q [G][hd] over the tokens
-    ``tok`` of one kv head; scale 1/sqrt(hd).  Returns [G][hd]."""
+    ``tok`` of one kv head; scale 1/sqrt(hd); ``bias`` an optional additive
+    mask over those tokens (0 or -inf).  Returns [G][hd]."""
     K = keys[tok]
     Vv = values[tok]
     s = q @ K.T / math.sqrt(q.shape[-1])
+    if bias is not None:
+        s = s + bias[None, :]
     s = s - s.max(axis=1, keepdims=True)
     p = np.exp(s)
     return (p @ Vv) / p.sum(axis=1, keepdims=True)
@@ -226,7 +235,7 @@ class Cache:
         self.n += c
 
 
-MODES = ("dense", "act", "kv", "both", "snap")
+MODES = ("dense", "act", "kv", "both", "snap", "masked")
 
 
 def decode_step(cfg, w, cache: Cache, token: int, mode: str, rp=1.0, rkv=1.0,
@@ -305,6 +314,12 @@ def decode_step(cfg, w, cache: Cache, token: int, mode: str, rp=1.0, rkv=1.0,
                                       for p in sel])
                 scores_l.append(sc)
                 pages_l.append(sel)
+            elif mode == "masked":
+                tok = np.arange(n_tok)
+                window = forced_pages(P, sinks, recent)
+                bias = np.where(np.isin(tok // page, sorted(window)), 0.0, -np.inf)
+                attn[h * G:(h + 1) * G] = attention(qg, keys, vals, tok, bias)
+                continue
             else:
                 tok = np.arange(n_tok)
             attn[h * G:(h + 1) * G] = attention(qg, keys, vals, tok)

@@ -168,3 +168,20 @@ def test_byte_account_rejects_bad_ratios():
     assert bc.bc_byte_account(C.byref(c), bc.BC_KV, 1.0, 0.0, 100, 1, 16, 16, C.byref(out)) == bc.BC_EINVAL
     assert bc.bc_byte_account(C.byref(c), bc.BC_ACT, 1.5, 1.0, 100, 1, 16, 16, C.byref(out)) == bc.BC_EINVAL
     assert bc.bc_byte_account(C.byref(c), bc.BC_KV, 1.0, 0.5, 100, 1, 0, 16, C.byref(out)) == bc.BC_EINVAL
+
+
+@pytest.mark.parametrize("n", [20463, 20464, 20479, 40959, 81919])
+@pytest.mark.parametrize("mode,rp,rkv", [("kv", 1.0, 0.3), ("both", 0.7, 0.3), ("snap", 1.0, 0.3),
+                                         ("kv", 1.0, 0.7), ("both", 0.3, 0.1)])
+def test_library_keep_counts_where_float_ratios_round_up(n, mode, rp, rkv):
+    """At P a multiple of 10 (1280, 2560, 5120 pages) r*P is an integer; the
+    library takes its ratios as doubles and keeps exactly the oracle's count
+    (a float32 ratio would keep one more page)."""
+    kw = dict(rp=rp, rkv=rkv, sinks=1, recent=16)
+    got = bc.byte_account(LLAMA_8B, mode, n, **kw)
+    ref = ba.implementation_bytes(LLAMA_8B, mode, n, **kw)
+    assert got["impl_kv_read_bytes"] == ref["kv_read"]
+    assert got["impl_total_bytes"] == ref["total"]
+    if mode != "snap":
+        P = -(-(n + 1) // 16)
+        assert got["pages_kept"] == ba.page_keep(P, rkv, 1, 16)[0]

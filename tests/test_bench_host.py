@@ -80,3 +80,36 @@ def test_site_labels_follow_the_projection_order():
         gemvs += "k_gemv" in nm
     assert sites == ["sel_qkv", "qkv", "page_scores", "page_select", "attn", "sel_o", "o", "sel_gate_up",
                      "gate_up", "sel_down", "down", "k_lmhead"]
+
+
+def test_crossing_of_first_sign_change():
+    assert bench.crossing_of([(0, -2.0), (10, -1.0), (20, 1.0), (30, -1.0)]) == pytest.approx(15.0)
+    assert bench.crossing_of([(0, 1.0), (10, 2.0)]) is None
+    assert bench.crossing_of([(0, -1.0), (10, 0.0)]) == pytest.approx(10.0)
+
+
+def test_sweep_fit_recovers_costs_and_predicts_every_pair():
+    """The sweep's cost-aware model (one bandwidth, a fixed cost per cell
+    kind) is recovered from cells built from it, its predicted crossing per
+    keep pair is where the model's act and kv times meet, and the crossing
+    measured on those cells by linear interpolation lies within one sweep
+    step of it."""
+    costs = {"dense": 1.30, "act@0.7": 1.80, "act": 1.90, "kv": 1.60, "kv@0.5": 1.55}
+    ctx = sorted(bench.SWEEP_CONTEXTS)
+    cells = {}
+    for c in bench.SWEEP_CELLS:
+        lib = bench.CELLS[c][0]
+        for n in ctx:
+            b = bc.byte_account(LLAMA_8B, lib, n, **bench.cell_kw(c))["impl_total_bytes"]
+            cells[(c, n)] = {"bytes_per_step": b, "ms_per_step": b / 6600e9 * 1e3 + costs[c]}
+    inv_bw, fitted = bench.cost_aware_fit(cells, ctx, bench.SWEEP_CELLS)
+    assert 1.0 / inv_bw == pytest.approx(6600.0, rel=1e-6)
+    for c, v in costs.items():
+        assert fitted[c] * 1e3 == pytest.approx(v, abs=1e-6)
+    for (rp, rkv), (ca, ck) in bench.CROSS_CELLS.items():
+        pred = bench.predicted_crossing(bc, LLAMA_8B, inv_bw, fitted, ca, ck)
+        meas = bench.crossing_of([(n, cells[(ca, n)]["ms_per_step"] - cells[(ck, n)]["ms_per_step"]) for n in ctx])
+        if pred is None or pred > max(ctx):
+            assert meas is None
+            continue
+        assert abs(meas - pred) <= 4096, (rp, rkv, meas, pred)

@@ -88,6 +88,28 @@ def test_kv_window_baseline(tiny):
                      to_host(logits), tr)
 
 
+def test_masked_dense_baseline(tiny):
+    """The masked dense baseline (every page read, an additive mask keeping
+    the window's pages) matches the oracle's masked step, and the KV window
+    computed from the window's pages alone, within fp32 rounding."""
+    cfg = tiny["cfg"]
+    kw = dict(sinks=1, recent=8)
+    m = _model(tiny)
+    cache = _cache(tiny)
+    logits = torch.empty(cfg["vocab"], device=DEV)
+    win = torch.empty(cfg["vocab"], device=DEV)
+    for tok in tokens(3, cfg["vocab"], seed=19):
+        n = len(m)
+        m.step(tok, "kv", win, rkv=1e-6, **kw)
+        m.reset(n)
+        m.step(tok, "masked", logits, **kw)
+        torch.cuda.synchronize()
+        tr = gpu_traces(m, cfg["n_layers"], False)
+        compare_step(cfg, tiny["wb"], cache, tok, "masked", 1.0, 1.0, kw["sinks"], kw["recent"],
+                     to_host(logits), tr)
+        assert max_rel(to_host(logits), to_host(win)) < 1e-5
+
+
 def test_keep_one_is_dense_bit_for_bit(tiny):
     cfg = tiny["cfg"]
     m = _model(tiny)
@@ -309,7 +331,7 @@ def big():
     return dict(cfg=cfg, wd=w, wb=wb, k=k, v=v, kb=bits(k), vb=bits(v))
 
 
-@pytest.mark.parametrize("mode", ["dense", "act", "kv", "both"])
+@pytest.mark.parametrize("mode", ["dense", "act", "kv", "both", "masked"])
 def test_llama8b_shape_step(big, mode):
     """One step at the Llama-3.1-8B shape (2048 cached tokens): every set
     exact on the GPU's own scores and within near-ties of the oracle's own

@@ -147,6 +147,26 @@ def test_attention_matches_sdpa():
     np.testing.assert_allclose(got, ref[0, :, 0].numpy(), rtol=1e-12, atol=1e-13)
 
 
+def test_attention_with_additive_mask_matches_sdpa_boolean_mask():
+    """The masked dense baseline's attention: an additive 0/-inf bias over
+    every token equals SDPA with a boolean mask, and attention over the kept
+    tokens alone."""
+    G, hd, T = 4, 32, 80
+    q = RNG.standard_normal((G, hd))
+    k = RNG.standard_normal((T, hd)) * 2
+    v = RNG.standard_normal((T, hd))
+    keep = np.zeros(T, dtype=bool)
+    keep[:16] = True
+    keep[48:] = True
+    bias = np.where(keep, 0.0, -np.inf)
+    got = od.attention(q, k, v, np.arange(T), bias)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[None, :, None, :], torch.from_numpy(k)[None, None].expand(1, G, -1, -1),
+        torch.from_numpy(v)[None, None].expand(1, G, -1, -1), attn_mask=torch.from_numpy(keep)[None, None, None])
+    np.testing.assert_allclose(got, ref[0, :, 0].numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(got, od.attention(q, k, v, np.flatnonzero(keep)), rtol=1e-12, atol=1e-13)
+
+
 def test_gemv_rows_matches_dense_and_masked():
     w = bf16_bits(torch.randn(40, 24).to(torch.bfloat16))
     x = RNG.standard_normal(40)
@@ -324,6 +344,23 @@ def test_both_composes_the_branches(tiny):
     for l in range(cfg["n_layers"]):
         for a, b in zip(tb[l]["pages"], tk[l]["pages"]):
             np.testing.assert_array_equal(a, b)
+
+
+def test_masked_dense_baseline_is_the_window(tiny):
+    """The masked dense baseline computes the KV window (sinks and recent
+    pages): it matches the kv mode with a keep ratio that leaves K = |F|."""
+    cfg, _, w, kb, vb = tiny
+    tok = tokens(6, cfg["vocab"], seed=5)[5]
+    kw = dict(sinks=1, recent=2)
+    masked, _ = _oracle(cfg, w, kb, vb, N_CTX, tok, "masked", **kw)
+    window, tw = _oracle(cfg, w, kb, vb, N_CTX, tok, "kv", rkv=1e-6, **kw)
+    P = -(-(N_CTX + 1) // 16)
+    for l in range(cfg["n_layers"]):
+        for sel in tw[l]["pages"]:
+            assert set(sel.tolist()) == od.forced_pages(P, 1, 2)
+    assert np.abs(masked - window).max() <= 1e-12 * np.abs(window).max()
+    dense, _ = _oracle(cfg, w, kb, vb, N_CTX, tok, "dense")
+    assert np.abs(masked - dense).max() > 1e-3 * np.abs(dense).max()
 
 
 def test_appended_kv_is_rounded_to_bf16(tiny):

@@ -38,8 +38,8 @@ def test_noalloc_matches_gemv_twice(d_in, d_out, k):
         got = torch.full((d_out,), float("nan"), device=DEV)
         bc.gemv_noalloc(W, x, idx, got)
         torch.cuda.synchronize()
-        err = (got - ref).abs().max().item() / ref.abs().max().item()
-        assert err <= 1e-5, err               # same kernel and plan: agrees to fp32 rounding
+        # the same deterministic kernel with the same plan on the same inputs: bit for bit
+        assert torch.equal(got, ref)
         assert np.isfinite(got.cpu().numpy()).all()
 
 
