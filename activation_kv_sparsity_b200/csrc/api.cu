@@ -947,6 +947,7 @@ extern "C" bc_status bc_attention(const float* q, const void* kv, int n_kv_heads
                                   int Pmax, const int* pages, int n_pages, int n_tok, float* out,
                                   void* scratch, size_t scratch_bytes, void* stream) {
   if (!q || !kv || !out || !scratch) return fail(BC_EINVAL, "null pointer");
+  if (((uintptr_t)q | (uintptr_t)kv | (uintptr_t)out) & 15) return fail(BC_EINVAL, "q, kv and out must be 16-byte aligned");
   if (head_dim != 64 && head_dim != 128) return fail(BC_EINVAL, "head_dim must be 64 or 128");
   if (n_kv_heads < 1 || group < 1 || group > 8) return fail(BC_EINVAL, "bad head counts");
   if (n_tok < 1 || n_pages < 1 || Pmax < n_pages || (n_tok + kPage - 1) / kPage > Pmax)

@@ -37,6 +37,7 @@
 #include "kernels.h"
 
 #include <algorithm>
+#include <type_traits>
 
 namespace bc {
 
@@ -77,26 +78,19 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn(AttnArgs a) {
   pdl_wait();
   pdl_trigger();
 
-  // A fragments of the queries, pre-scaled to base-2 logits
+  // This lane's query values: k-step s contracts dims (s/2)*32 + t*8 +
+  // 4*(s%2) + 0..3.  They are loaded here and turned into A fragments only
+  // after the first page's loads are issued, so the two latencies overlap.
   const float qscale = 1.4426950408889634f * rsqrtf((float)HD);
-  uint32_t qa[KSTEPS][4];
+  float4 qraw[KSTEPS];
   {
     const float* qrow = a.q + (size_t)(h * G + g) * HD + t * 8;
     #pragma unroll
-    for (int s = 0; s < KSTEPS; ++s) {
-      // k-step s contracts dims (s/2)*32 + t*8 + 4*(s%2) + 0..3 of this lane
-      const int d0 = (s / 2) * 32 + 4 * (s % 2);
-      float q0 = 0.f, q1 = 0.f, q2 = 0.f, q3 = 0.f;
-      if (g < G) {
-        q0 = qrow[d0] * qscale;
-        q1 = qrow[d0 + 1] * qscale;
-        q2 = qrow[d0 + 2] * qscale;
-        q3 = qrow[d0 + 3] * qscale;
-      }
-      split2(q0, q1, qa[s][0], qa[s][1]);
-      split2(q2, q3, qa[s][2], qa[s][3]);
-    }
+    for (int s = 0; s < KSTEPS; ++s)
+      qraw[s] = g < G ? *reinterpret_cast<const float4*>(qrow + (s / 2) * 32 + 4 * (s % 2))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  uint32_t qa[KSTEPS][4];
 
   float o[NBLK][4];
   #pragma unroll
@@ -222,6 +216,12 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn(AttnArgs a) {
     pa_cur = page_of(0);
     load_page(pa_cur, ka0, ka1, va0, va1);
   }
+  // A fragments of the queries, pre-scaled to base-2 logits
+  #pragma unroll
+  for (int s = 0; s < KSTEPS; ++s) {
+    split2(qraw[s].x * qscale, qraw[s].y * qscale, qa[s][0], qa[s][1]);
+    split2(qraw[s].z * qscale, qraw[s].w * qscale, qa[s][2], qa[s][3]);
+  }
   for (int jj = 0; jj < n_it;) {
     advance(jj);
     prefetch(jj + 2);
@@ -278,74 +278,74 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn(AttnArgs a) {
     }
   }
 
-  // the last split of this kv head to finish merges the partials
+  // The last split CTA of this kv head to finish merges the partials.  The
+  // barrier orders the CTA's partial stores before thread 0's release
+  // increment of the ticket; the last CTA's acquire orders its reads after
+  // every other CTA's stores.
   __shared__ int s_last;
-  __shared__ float s_w[8][kMaxSplits];
-  __shared__ float s_inv[8];
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(&a.counters[h], 1u) == (unsigned)(a.splits - 1));
+  if (threadIdx.x == 0) {
+    unsigned prev;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(prev) : "l"(a.counters + h) : "memory");
+    s_last = prev == (unsigned)(a.splits - 1);
+  }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   if (threadIdx.x == 0) a.counters[h] = 0u;
-  __shared__ float s_l2[8][kMaxSplits];
-  #pragma unroll 4
-  for (int e = threadIdx.x; e < G * kMaxSplits; e += kAttnWarps * 32) {
-    const int hh = e / kMaxSplits, sp = e % kMaxSplits;
-    float m = -INFINITY, l = 0.f;
-    if (sp < a.splits) {
-      const float2 ml = *reinterpret_cast<const float2*>(&a.part_ml[((size_t)(h * G + hh) * kMaxSplits + sp) * 2]);
-      m = ml.x;
-      l = ml.y;
-    }
-    s_w[hh][sp] = m;
-    s_l2[hh][sp] = l;
-  }
-  __syncthreads();
-  // one warp per head: max, weights and normaliser over the splits
-  for (int hh = threadIdx.x >> 5; hh < G; hh += kAttnWarps) {
-    const int ln = threadIdx.x & 31;
-    float M = -INFINITY;
-    for (int sp = ln; sp < a.splits; sp += 32) M = fmaxf(M, s_w[hh][sp]);
+  // One warp per query head of the group; lane l owns dims DPL2*l .. +DPL2.
+  // Each lane issues the splits' (m, l) and its own slice of their outputs
+  // together (up to kComb splits in flight), so the merge costs one round
+  // trip to L2 per kComb splits: o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+  constexpr int DPL2 = HD / 32;
+  constexpr int kComb = 40;
+  using vec_t = typename std::conditional<DPL2 == 4, float4, float2>::type;
+  for (int hh = warp; hh < G; hh += kAttnWarps) {
+    const int qh = h * G + hh;
+    const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + (size_t)qh * kMaxSplits;
+    const vec_t* po = reinterpret_cast<const vec_t*>(a.part_o + (size_t)qh * kMaxSplits * HD) + lane;
+    float acc[DPL2];
     #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.f;
-    for (int sp = ln; sp < kMaxSplits; sp += 32) {
-      const float m = s_w[hh][sp];
-      const float w = (sp < a.splits && m != -INFINITY) ? exp2f(m - M) : 0.f;
-      s_w[hh][sp] = w;
-      L += w * s_l2[hh][sp];
-    }
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (ln == 0) s_inv[hh] = 1.0f / L;
-  }
-  __syncthreads();
-  // each thread owns 4 consecutive outputs (a float4) and sums the splits in
-  // order, up to 32 split loads in flight at a time
-  constexpr int kFly = 32;
-  for (int e4 = threadIdx.x; e4 < G * HD / 4; e4 += kAttnWarps * 32) {
-    const int hh = (e4 * 4) / HD, d = (e4 * 4) % HD;
-    const float4* po = reinterpret_cast<const float4*>(a.part_o + (size_t)(h * G + hh) * kMaxSplits * HD + d);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int sp0 = 0; sp0 < a.splits; sp0 += kFly) {
-      float4 v[kFly];
+    for (int d = 0; d < DPL2; ++d) acc[d] = 0.f;
+    float M = -INFINITY, L = 0.f;
+    for (int sp0 = 0; sp0 < a.splits; sp0 += kComb) {
+      const int nsp = min(kComb, a.splits - sp0);
+      vec_t ov[kComb];
       #pragma unroll
-      for (int u = 0; u < kFly; ++u)
-        v[u] = sp0 + u < a.splits ? __ldcg(po + (size_t)(sp0 + u) * (HD / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int u = 0; u < kComb; ++u)
+        if (u < nsp) ov[u] = __ldcg(po + (size_t)(sp0 + u) * (HD / DPL2));
+      // (m, l) of splits sp0 + lane and sp0 + 32 + lane
+      float2 m0 = make_float2(-INFINITY, 0.f), m1 = m0;
+      if (lane < nsp) m0 = __ldcg(ml + sp0 + lane);
+      if (32 + lane < nsp) m1 = __ldcg(ml + sp0 + 32 + lane);
+      float cm = fmaxf(m0.x, m1.x);
       #pragma unroll
-      for (int u = 0; u < kFly; ++u) {
-        const float w = sp0 + u < a.splits ? s_w[hh][sp0 + u] : 0.f;
-        acc.x += w * v[u].x;
-        acc.y += w * v[u].y;
-        acc.z += w * v[u].z;
-        acc.w += w * v[u].w;
+      for (int o = 16; o > 0; o >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o));
+      const float M_new = fmaxf(M, cm);
+      const float base2 = M_new == -INFINITY ? 0.f : M_new;
+      const float w0 = m0.x == -INFINITY ? 0.f : exp2f(m0.x - base2);
+      const float w1 = m1.x == -INFINITY ? 0.f : exp2f(m1.x - base2);
+      float cl = w0 * m0.y + w1 * m1.y;
+      #pragma unroll
+      for (int o = 16; o > 0; o >>= 1) cl += __shfl_xor_sync(0xffffffffu, cl, o);
+      const float scale = M == -INFINITY ? 0.f : exp2f(M - base2);
+      L = L * scale + cl;
+      #pragma unroll
+      for (int d = 0; d < DPL2; ++d) acc[d] *= scale;
+      #pragma unroll
+      for (int u = 0; u < kComb; ++u) {
+        if (u < nsp) {
+          const float w = __shfl_sync(0xffffffffu, u < 32 ? w0 : w1, u & 31);
+          const float* ovf = reinterpret_cast<const float*>(&ov[u]);
+          #pragma unroll
+          for (int d = 0; d < DPL2; ++d) acc[d] = fmaf(w, ovf[d], acc[d]);
+        }
       }
+      M = M_new;
     }
-    const float inv = s_inv[hh];
-    *reinterpret_cast<float4*>(a.out + (size_t)(h * G + hh) * HD + d) =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    const float inv = 1.0f / L;
+    float* dst = a.out + (size_t)qh * HD + lane * DPL2;
+    #pragma unroll
+    for (int d = 0; d < DPL2; ++d) dst[d] = acc[d] * inv;
   }
 }
 

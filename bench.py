@@ -237,9 +237,15 @@ def run_ours(args, rank, ws, local):
     max_ctx = max(contexts + sweep_ctx) + warm + steps + 32
     w = make_weights(cfg, seed=0, device=dev)
     model = bc.Model(cfg, w, max_ctx)
-    for k, v in kv_chunks(cfg, max(contexts + sweep_ctx), seed=1, device=dev):
-        model.append(k, v)
-    torch.cuda.synchronize()
+
+    def refill():
+        # the synthetic cache up to the longest context (each pass over the
+        # contexts runs from long to short, so every cell reads pristine KV)
+        model.reset(0)
+        for k, v in kv_chunks(cfg, max(contexts + sweep_ctx), seed=1, device=dev):
+            model.append(k, v)
+        torch.cuda.synchronize()
+    refill()
     stream = model.stream
     logits = torch.empty(cfg["vocab"], device=dev)
     toks = [(1 + 7919 * i) % cfg["vocab"] for i in range(warm + steps)]
@@ -345,6 +351,7 @@ def run_ours(args, rank, ws, local):
     # the crossing sweep: blocks of every sweep cell at every context
     sweep = []
     for b in range(args.sweep_blocks):
+        refill()
         block = {}
         for n in sweep_ctx:
             for name in SWEEP_CELLS:
@@ -366,18 +373,13 @@ def run_ours(args, rank, ws, local):
     y = torch.empty(d_out, device=dev)
     scratch = torch.zeros(bc.bc_gemv_scratch_bytes(d_out), dtype=torch.uint8, device=dev)
     wgu = w["wgu_t"]
-    for l in range(4):
-        bc.gemv(wgu[l], xin, idx, y, scratch, stream)
-    torch.cuda.synchronize()
-    reps = 4
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        for l in range(cfg["n_layers"]):
-            bc.gemv(wgu[l], xin, idx, y, scratch, stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    gemv_ms = e0.elapsed_time(e1) / (reps * cfg["n_layers"])
+    it = [0]
+
+    def launch_gu():
+        bc.gemv(wgu[it[0] % cfg["n_layers"]], xin, idx, y, scratch)
+        it[0] += 1
+    # 4 x 32 launches over the 32 layers' weights, replayed from a CUDA graph
+    gemv_ms = graph_timed(launch_gu, 4, 4 * cfg["n_layers"], dev)
     gemv_bytes = kq * d_out * 2 + kq * 8            # weight rows + index/activation reads
     achieved = gemv_bytes / (gemv_ms * 1e-3) / 1e9
 
@@ -677,6 +679,33 @@ def run_reference(args, rank, ws, local):
     }
 
 
+def graph_timed(launch, warmup, steps, dev):
+    """Milliseconds per launch of `steps` back-to-back launches replayed
+    from one CUDA graph (no host launch cost between them), after `warmup`
+    direct launches.  launch() must enqueue on the current stream."""
+    import torch
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        for _ in range(warmup):
+            launch()
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for _ in range(steps):
+            launch()
+    gr.replay()
+    torch.cuda.synchronize()
+    cur = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    gr.replay()
+    e1.record(cur)
+    torch.cuda.synchronize()
+    del gr
+    return e0.elapsed_time(e1) / steps
+
+
 def run_kernel_only(args, local):
     """Times one kernel alone on a small case (for profiler captures): the
     gathered gate/up GEMV of one layer (235 MB dense, 117 MB at rp 0.5) or
@@ -734,7 +763,44 @@ def run_kernel_only(args, local):
         nbytes = k * d_out * 2 + k * 8
 
         def launch():
-            bc.gemv(W, x, idx, y, scratch, stream)
+            bc.gemv(W, x, idx, y, scratch)
+    elif args.only_kernel in ("select", "select_wide"):
+        # the exact top-k of the projection branch alone: 2048 of 4096
+        # (q/k/v, o, gate/up inputs) or 7168 of 14336 (the down input)
+        n = 4096 if args.only_kernel == "select" else 14336
+        k = math.ceil(0.5 * n - 1e-9)
+        vs = torch.randn(64, n, generator=g, device=dev)
+        idx = torch.empty(k, dtype=torch.int32, device=dev)
+        nbytes = 0
+        it = [0]
+
+        def launch():
+            bc.select_topk(vs[it[0] % 64], k, idx)
+            it[0] += 1
+    elif args.only_kernel == "attention_short":
+        # the both@32K attention: 615 of 2049 pages per kv head (the sink,
+        # the 16 recent pages and 598 others), 8 layers' pools in turn so
+        # that no launch finds its pages in L2 (40 MB a launch, 1.07 GB of pools)
+        Hkv, G, hd, n_tok, nl = cfg["n_kv_heads"], cfg["n_heads"] // cfg["n_kv_heads"], cfg["head_dim"], 32769, 8
+        P = -(-n_tok // 16)
+        K = math.ceil(0.3 * P - 1e-9)
+        pools = torch.randn(nl, Hkv, P, 2, 16, hd, generator=g, device=dev).to(torch.bfloat16)
+        lists = torch.zeros(nl, Hkv, P, dtype=torch.int32, device=dev)
+        for l in range(nl):
+            for h in range(Hkv):
+                mid = torch.randperm(P - 17, generator=g, device=dev)[:K - 17] + 1
+                sel = torch.cat([torch.tensor([0], device=dev), mid, torch.arange(P - 16, P, device=dev)])
+                lists[l, h, :K] = torch.sort(sel)[0].to(torch.int32)
+        q = torch.randn(Hkv * G, hd, generator=g, device=dev)
+        out = torch.empty(Hkv * G, hd, device=dev)
+        scratch = torch.zeros(bc.bc_attention_scratch_bytes(Hkv * G, hd), dtype=torch.uint8, device=dev)
+        nbytes = Hkv * (K * 16 - (P * 16 - n_tok)) * 2 * hd * 2
+        it = [0]
+
+        def launch():
+            l = it[0] % nl
+            it[0] += 1
+            bc.attention(q, pools[l], Hkv, G, hd, P, lists[l], K, n_tok, out, scratch)
     else:
         Hkv, G, hd, n_tok = cfg["n_kv_heads"], cfg["n_heads"] // cfg["n_kv_heads"], cfg["head_dim"], 131073
         P = -(-n_tok // 16)
@@ -745,22 +811,16 @@ def run_kernel_only(args, local):
         nbytes = Hkv * n_tok * 2 * hd * 2
 
         def launch():
-            bc.attention(q, pool, Hkv, G, hd, P, None, P, n_tok, out, scratch, stream)
-    for _ in range(args.warmup):
-        launch()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        launch()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
+            bc.attention(q, pool, Hkv, G, hd, P, None, P, n_tok, out, scratch)
+    ms = graph_timed(launch, args.warmup, args.steps, dev)
     peak, kind = peaks()
+    if not nbytes:
+        return {"kernel": args.only_kernel, "us_per_launch": round(ms * 1e3, 3),
+                "note": "launches back to back on one stream (programmatic dependent launch)"}
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"kernel": args.only_kernel, "ms_per_launch": round(ms, 5), "algorithmic_bytes": nbytes,
             "gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "peak": peak, "peak_kind": kind,
-            "note": "includes the combine kernel" if args.only_kernel == "attention" else ""}
+            "note": "includes the fused combine" if args.only_kernel.startswith("attention") else ""}
 
 
 def run_batch_gemv(args, dev, stream, cfg):
@@ -910,7 +970,8 @@ def main():
                     help="per-site cost of one step in this mode at the first --contexts value")
     ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",
                     help="write profiles/traffic.json from an ncu raw CSV of --only-kernel gemv_gateup")
-    ap.add_argument("--only-kernel", choices=("gemv_gateup", "gemv_gateup_dense", "attention", "snap", "gemv_batch"),
+    ap.add_argument("--only-kernel", choices=("gemv_gateup", "gemv_gateup_dense", "attention", "attention_short", "snap",
+                                              "gemv_batch", "select", "select_wide"),
                     help="time one kernel alone on a small case (profiler captures)")
     args = ap.parse_args()
     if args.record_traffic:

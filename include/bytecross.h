@@ -315,7 +315,8 @@ BC_API bc_status bc_select_topk(const float* v, int n, int k, int* idx, void* st
 
 /* Split-K flash-decode attention of one layer over a page list, the
  * attention kernel of every mode (README, "Overview").
- *   q      device f32 [Hkv*G][hd] rotated queries (G query heads per kv head)
+ *   q      device f32 [Hkv*G][hd] rotated queries (G query heads per kv head);
+ *          q, kv and out 16-byte aligned (else BC_EINVAL)
  *   kv     device bf16 pages of one layer, [Hkv][Pmax][2][16][hd]
  *   pages  device int32 [Hkv][Pmax] kept pages per kv head (first n_pages of
  *          each row used, ascending), or NULL for pages 0..n_pages-1
