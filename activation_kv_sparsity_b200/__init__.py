@@ -77,6 +77,19 @@ _SIGS = {
                                   C.c_int, C.c_int, C.POINTER(bc_bytes)]),
     "bc_crossover_batch": (C.c_int, [C.POINTER(bc_config), C.c_double, C.c_double, C.c_int,
                                      C.POINTER(C.c_double)]),
+    "bc_batch_workspace_bytes": (C.c_size_t, [C.POINTER(bc_config), C.c_int]),
+    "bc_batch_create": (C.c_int, [C.POINTER(bc_config), C.POINTER(bc_weights), C.c_int, _P, _P, _P, C.c_size_t, _P,
+                                  C.POINTER(_P)]),
+    "bc_batch_destroy": (C.c_int, [_P]),
+    "bc_batch_set_graphs": (C.c_int, [_P, C.c_int]),
+    "bc_batch_length": (C.c_int, [_P]),
+    "bc_batch_launch_count": (C.c_longlong, [_P]),
+    "bc_batch_reset": (C.c_int, [_P, C.c_int]),
+    "bc_batch_append": (C.c_int, [_P, _P, _P, C.c_int]),
+    "bc_batch_step": (C.c_int, [_P, C.POINTER(C.c_int), C.c_int, C.c_double, C.c_double, C.c_int, C.c_int, C.c_int,
+                                _P]),
+    "bc_batch_trace": (C.c_int, [_P, C.c_int, C.c_int, C.c_int, C.POINTER(_P), C.POINTER(C.c_int),
+                                 C.POINTER(C.c_int)]),
     "bc_last_error": (C.c_char_p, []),
     "bc_status_string": (C.c_char_p, [C.c_int]),
 }
@@ -211,6 +224,96 @@ class Model:
             t = self.workspace[off:off + 4 * rows * stride.value].view(dt).view(rows, stride.value)
             return t[:, :cnt.value]
         return self.workspace[off:off + 4 * cnt.value].view(dt)
+
+
+_INT_TRACES = (BC_TRACE_SEL_QKV, BC_TRACE_SEL_O, BC_TRACE_SEL_GU, BC_TRACE_SEL_D, BC_TRACE_PAGES, BC_TRACE_SNAP_PAGES)
+
+
+class Batch:
+    """A batch of sequences decoding in lock step (bc_batch_*): owns the
+    sequences' KV and bound pools and the workspace (allocated with torch)."""
+
+    def __init__(self, cfg: dict, weights: dict, batch: int, max_ctx: int, stream=None):
+        import torch
+        self.cfg = cfg
+        self.B = batch
+        self.c = config(cfg, max_ctx)
+        self.weights = weights
+        dev = weights["embed"].device
+        self.stream = stream if stream is not None else torch.cuda.current_stream(dev)
+        kvb = bc_kv_pool_bytes(C.byref(self.c))
+        mb = bc_meta_pool_bytes(C.byref(self.c))
+        wsb = bc_batch_workspace_bytes(C.byref(self.c), batch)
+        if not (kvb and mb and wsb):
+            raise ValueError("bad config or batch size for a libbytecross batch")
+        self.kv_pool = torch.empty(batch * kvb, dtype=torch.uint8, device=dev)
+        self.meta_pool = torch.empty(batch * mb, dtype=torch.uint8, device=dev)
+        self.workspace = torch.zeros(wsb, dtype=torch.uint8, device=dev)
+        w = bc_weights(*(C.c_void_p(weights[k].data_ptr()) for k in (
+            "embed", "lm_head", "final_norm", "attn_norm", "mlp_norm", "wqkv_t", "wo_t", "wgu_t", "wd_t")))
+        h = C.c_void_p()
+        check(bc_batch_create(C.byref(self.c), C.byref(w), batch, C.c_void_p(self.kv_pool.data_ptr()),
+                              C.c_void_p(self.meta_pool.data_ptr()), C.c_void_p(self.workspace.data_ptr()), wsb,
+                              C.c_void_p(self.stream.cuda_stream), C.byref(h)), "bc_batch_create")
+        self.h = h
+
+    def close(self):
+        if getattr(self, "h", None):
+            bc_batch_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __len__(self):
+        return bc_batch_length(self.h)
+
+    def set_graphs(self, enable: bool):
+        check(bc_batch_set_graphs(self.h, 1 if enable else 0), "bc_batch_set_graphs")
+
+    def launches(self) -> int:
+        return bc_batch_launch_count(self.h)
+
+    def reset(self, n_ctx: int):
+        check(bc_batch_reset(self.h, n_ctx), "bc_batch_reset")
+
+    def append(self, k, v):
+        """k, v: bf16 device tensors [batch][L][Hkv][n][hd]."""
+        k, v = k.contiguous(), v.contiguous()
+        check(bc_batch_append(self.h, C.c_void_p(k.data_ptr()), C.c_void_p(v.data_ptr()), k.shape[3]),
+              "bc_batch_append")
+
+    def step(self, tokens, mode: str, logits, rp=1.0, rkv=1.0, sinks=1, recent=16):
+        """tokens: B ints; logits: f32 device tensor [B][vocab]."""
+        toks = (C.c_int * self.B)(*[int(t) for t in tokens])
+        check(bc_batch_step(self.h, toks, MODES[mode], rp, rkv, sinks, recent, self.c.page,
+                            C.c_void_p(logits.data_ptr())), "bc_batch_step")
+
+    def seq(self, b: int):
+        """A view of sequence b with the trace() of a Model."""
+        return _BatchSeq(self, b)
+
+
+class _BatchSeq:
+    def __init__(self, batch: Batch, b: int):
+        self.batch, self.b, self.cfg = batch, b, batch.cfg
+
+    def trace(self, layer: int, kind: int):
+        import torch
+        bt = self.batch
+        ptr, cnt, stride = C.c_void_p(), C.c_int(), C.c_int()
+        check(bc_batch_trace(bt.h, self.b, layer, kind, C.byref(ptr), C.byref(cnt), C.byref(stride)),
+              "bc_batch_trace")
+        off = ptr.value - bt.workspace.data_ptr()
+        dt = torch.int32 if kind in _INT_TRACES else torch.float32
+        if stride.value:
+            rows = self.cfg["n_kv_heads"]
+            t = bt.workspace[off:off + 4 * rows * stride.value].view(dt).view(rows, stride.value)
+            return t[:, :cnt.value]
+        return bt.workspace[off:off + 4 * cnt.value].view(dt)
 
 
 # ------------------------------------------------------------------ single kernels

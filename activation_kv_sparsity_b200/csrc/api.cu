@@ -389,6 +389,7 @@ static cudaError_t step_select(bc_model* m, int prep, int n, int k, const float*
                                const __nv_bfloat16* gain, const __nv_bfloat16* emb, float* x_init,
                                float* vout, int* idx, SelectArgs* out_args) {
   SelectArgs s;
+  memset(&s, 0, sizeof s);
   s.prep = prep;
   s.n = n;
   s.k = k;

@@ -60,6 +60,16 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn(AttnArgs a) {
   __shared__ float s_o[kAttnWarps][8][HD];
   __shared__ float s_m[kAttnWarps][8], s_l[kAttnWarps][8];
 
+  if (blockIdx.z) {                               // batched launch: sequence blockIdx.z
+    const long long b = blockIdx.z;
+    a.q += b * a.q_stride;
+    a.kv += b * a.kv_stride;
+    if (a.pages) a.pages += b * a.list_stride;
+    a.part_o += b * a.part_stride * HD;
+    a.part_ml += b * a.part_stride * 2;
+    a.counters += b * a.counters_stride;
+    a.out += b * a.out_stride;
+  }
   const int split = blockIdx.x, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -375,9 +385,9 @@ static cudaError_t launch_k(K kern, dim3 grid, dim3 block, cudaStream_t st, bool
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st, bool pdl) {
-  if (a.hd == 128) return launch_k(k_attn<128>, dim3(a.splits, a.Hkv), dim3(kAttnWarps * 32), st, pdl, a);
-  if (a.hd == 64) return launch_k(k_attn<64>, dim3(a.splits, a.Hkv), dim3(kAttnWarps * 32), st, pdl, a);
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st, bool pdl, int nb) {
+  if (a.hd == 128) return launch_k(k_attn<128>, dim3(a.splits, a.Hkv, nb), dim3(kAttnWarps * 32), st, pdl, a);
+  if (a.hd == 64) return launch_k(k_attn<64>, dim3(a.splits, a.Hkv, nb), dim3(kAttnWarps * 32), st, pdl, a);
   return cudaErrorInvalidValue;
 }
 

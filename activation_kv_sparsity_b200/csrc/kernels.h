@@ -66,8 +66,11 @@ struct SelectArgs {
   float* x_init;                  // EMBED_NORM: residual stream initialised here
   float* vout;                    // the ranked vector (trace), or nullptr
   int* idx;                       // [k] ascending
+  // batched launch (nb vectors, one per sequence): vector b is read from
+  // x + b*x_stride and ranked into idx + b*idx_stride (SP_NONE only)
+  long long x_stride, idx_stride;
 };
-cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl);
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl, int nb = 1);
 
 // ------------------------------------------------------------------ KV pages
 // Page scores (grid-wide), then the page select (one CTA, or above 8192
@@ -80,9 +83,13 @@ struct PageArgs {
   float* scores;                  // [Hkv][Pmax]
   int* pages;                     // [Hkv][Pmax], first K ascending
   unsigned* counters;             // unused (kept for the workspace layout)
+  // batched launch (nb sequences of equal length): sequence b's queries,
+  // bounds, scores and pages are at q + b*q_stride, meta + b*meta_stride,
+  // scores / pages + b*sp_stride (elements)
+  long long q_stride, meta_stride, sp_stride;
 };
-cudaError_t launch_page_scores(const PageArgs& a, cudaStream_t st, bool pdl);
-cudaError_t launch_page_select(const PageArgs& a, cudaStream_t st, bool pdl);
+cudaError_t launch_page_scores(const PageArgs& a, cudaStream_t st, bool pdl, int nb = 1);
+cudaError_t launch_page_select(const PageArgs& a, cudaStream_t st, bool pdl, int nb = 1);
 // Which page-select kernel P pages take: keys per thread of the one-CTA
 // kernel (2, 4 or 8), or 0 for the cluster.  A captured step serves only
 // page counts of its own variant.
@@ -120,9 +127,13 @@ struct AttnArgs {
   float* part_ml;                 // [Hkv*G][kMaxSplits][2]
   unsigned* counters;             // [Hkv], zero between launches
   float* out;                     // [Hkv*G][hd]
+  // batched launch (nb sequences of equal length): sequence b's tensors are
+  // offset by b times these strides (elements)
+  long long q_stride, kv_stride, list_stride, part_stride, out_stride;
+  int counters_stride;
 };
 void attn_plan(int n_pages, int Hkv, int sms, int* splits, int* pps);
-cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st, bool pdl);
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t st, bool pdl, int nb = 1);
 
 // ------------------------------------------------------------------ KV append (bulk)
 struct KvAppendArgs {

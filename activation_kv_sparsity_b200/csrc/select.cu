@@ -158,6 +158,8 @@ __device__ void cluster_topk(const uint32_t* s_key, int s0, int ns, int need, St
 }
 
 __global__ void __launch_bounds__(kSelClThreads, 1) k_select(SelectArgs a) {
+  a.x += blockIdx.y * a.x_stride;                 // batched launch: vector blockIdx.y
+  a.idx += blockIdx.y * a.idx_stride;
   __shared__ uint32_t s_key[kSelSlice];
   __shared__ SelClusterSmem sm;
   cg::cluster_group cl = cg::this_cluster();
@@ -219,6 +221,8 @@ constexpr int kSelThreads1 = 1024;
 
 template <int KPT>
 __global__ void __launch_bounds__(kSelThreads1, 1) k_select_cta(SelectArgs a) {
+  a.x += blockIdx.x * a.x_stride;                 // batched launch: vector blockIdx.x
+  a.idx += blockIdx.x * a.idx_stride;
   __shared__ RegTopkSmem<kSelThreads1> sm;
   const int tid = threadIdx.x, n = a.n;
   const int ibase = (tid >> 5) * KPT * 32 + (tid & 31);
@@ -259,10 +263,10 @@ __global__ void __launch_bounds__(kSelThreads1, 1) k_select_cta(SelectArgs a) {
   reg_topk<kSelThreads1, KPT>(kr, n, a.k, [](int) { return (uint8_t)ST_CAND; }, a.idx, sm);
 }
 
-cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl) {
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl, int nb) {
   cudaLaunchConfig_t cfg = {};
   if (a.n <= kSelOneCta) {
-    cfg.gridDim = dim3(1);
+    cfg.gridDim = dim3(nb);
     cfg.blockDim = dim3(kSelThreads1);
     cfg.stream = st;
     cudaLaunchAttribute attr1[1];
@@ -273,7 +277,7 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl) {
     if (a.n <= kSelThreads1 * 4) return cudaLaunchKernelEx(&cfg, k_select_cta<4>, a);
     return cudaLaunchKernelEx(&cfg, k_select_cta<8>, a);
   }
-  cfg.gridDim = dim3(kSelCluster);
+  cfg.gridDim = dim3(kSelCluster, nb);
   cfg.blockDim = dim3(kSelClThreads);
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
@@ -359,6 +363,9 @@ __host__ __device__ constexpr int pages_per_round() {
 
 template <int HD, int GMAX>
 __global__ void __launch_bounds__(kPageThreads, GMAX <= 4 ? 2 : 1) k_pages(PageArgs a) {
+  a.q += blockIdx.z * a.q_stride;                 // batched launch: sequence blockIdx.z
+  a.meta += blockIdx.z * a.meta_stride;
+  a.scores += blockIdx.z * a.sp_stride;
   constexpr int LPP = HD / 8;          // lanes per page
   constexpr int PPW = 32 / LPP;        // pages per warp step
   constexpr int STEPS = 4;             // warp steps per round
@@ -428,6 +435,8 @@ __global__ void __launch_bounds__(kPageThreads, GMAX <= 4 ? 2 : 1) k_pages(PageA
 // kept and not ranked.  (One 1024-thread CTA with 16 keys a thread measured
 // slower.)
 __global__ void __launch_bounds__(kSelClThreads, 1) k_page_select(PageArgs a) {
+  a.scores += blockIdx.z * a.sp_stride;           // batched launch: sequence blockIdx.z
+  a.pages += blockIdx.z * a.sp_stride;
   __shared__ uint32_t s_key[kSelSlice];
   __shared__ SelClusterSmem sm;
   cg::cluster_group cl = cg::this_cluster();
@@ -462,6 +471,8 @@ __global__ void __launch_bounds__(kSelClThreads, 1) k_page_select(PageArgs a) {
 // register keys (KPT per thread, P <= 1024*KPT), forced pages kept.
 template <int KPT>
 __global__ void __launch_bounds__(kSelThreads1, 1) k_page_select_cta(PageArgs a) {
+  a.scores += blockIdx.y * a.sp_stride;           // batched launch: sequence blockIdx.y
+  a.pages += blockIdx.y * a.sp_stride;
   __shared__ RegTopkSmem<kSelThreads1> sm;
   const int h = blockIdx.x, tid = threadIdx.x, P = a.P;
   const int ibase = (tid >> 5) * KPT * 32 + (tid & 31);
@@ -494,9 +505,10 @@ dim3 pages_grid(const PageArgs& a) {
   return dim3((a.P + ppc - 1) / ppc, a.Hkv);
 }
 
-cudaError_t launch_page_scores(const PageArgs& a, cudaStream_t st, bool pdl) {
+cudaError_t launch_page_scores(const PageArgs& a, cudaStream_t st, bool pdl, int nb) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = pages_grid(a);
+  cfg.gridDim.z = nb;
   cfg.blockDim = dim3(kPageThreads);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -517,7 +529,7 @@ int page_select_variant(int P) {
   return 0;
 }
 
-cudaError_t launch_page_select(const PageArgs& a, cudaStream_t st, bool pdl) {
+cudaError_t launch_page_select(const PageArgs& a, cudaStream_t st, bool pdl, int nb) {
   cudaLaunchConfig_t cfg = {};
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
@@ -525,7 +537,7 @@ cudaError_t launch_page_select(const PageArgs& a, cudaStream_t st, bool pdl) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   const int variant = page_select_variant(a.P);
   if (variant) {
-    cfg.gridDim = dim3(a.Hkv);
+    cfg.gridDim = dim3(a.Hkv, nb);
     cfg.blockDim = dim3(kSelThreads1);
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
@@ -533,7 +545,7 @@ cudaError_t launch_page_select(const PageArgs& a, cudaStream_t st, bool pdl) {
     if (variant == 4) return cudaLaunchKernelEx(&cfg, k_page_select_cta<4>, a);
     return cudaLaunchKernelEx(&cfg, k_page_select_cta<8>, a);
   }
-  cfg.gridDim = dim3(kSelCluster, a.Hkv);
+  cfg.gridDim = dim3(kSelCluster, a.Hkv, nb);
   cfg.blockDim = dim3(kSelClThreads);
   attr[1].id = cudaLaunchAttributeClusterDimension;
   attr[1].val.clusterDim.x = kSelCluster;

@@ -359,6 +359,43 @@ def run_ours(args, rank, ws, local):
                 block[(name, n)] = {"ms_per_step": ms, "bytes_per_step": step_bytes(name, n, sw_steps)[1]}
         sweep.append(block)
 
+    # the batched step: B sequences of equal length in lock step, each with
+    # its own cache, against B batch-1 steps of the same context and mode
+    batch_rows = []
+    if args.batch_ctx and args.batch_ctx in contexts:
+        n_b = args.batch_ctx
+        for B in args.batches:
+            bt = bc.Batch(cfg, w, B, n_b + warm + steps + 8)
+            chunks = [list(kv_chunks(cfg, n_b, seed=1 + b, device=dev)) for b in range(B)]
+            for i in range(len(chunks[0])):
+                bt.append(torch.stack([chunks[b][i][0] for b in range(B)]),
+                          torch.stack([chunks[b][i][1] for b in range(B)]))
+            del chunks
+            blog = torch.empty(B, cfg["vocab"], device=dev)
+            for name in ("act", "both"):
+                lib, kw = CELLS[name]
+                bt.reset(n_b)
+                for i in range(warm):
+                    bt.step([(toks[i] + b) % cfg["vocab"] for b in range(B)], lib, blog, **kw)
+                torch.cuda.synchronize()
+                l0 = bt.launches()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(bt.stream)
+                for i in range(steps):
+                    bt.step([(toks[warm + i] + b) % cfg["vocab"] for b in range(B)], lib, blog, **kw)
+                e1.record(bt.stream)
+                torch.cuda.synchronize()
+                ms = e0.elapsed_time(e1) / steps
+                t1 = cells[(name, n_b)]["ms_per_step"] if (name, n_b) in cells else None
+                batch_rows.append({"batch": B, "mode": name, "context": n_b, "ms_per_step": round(ms, 4),
+                                   "tok_s": round(1000.0 * B / ms, 2),
+                                   "ms_per_step_batch1": t1,
+                                   "speedup_vs_separate_steps": round(B * t1 / ms, 3) if t1 else None,
+                                   "launches_per_step": (bt.launches() - l0) // steps})
+            bt.close()
+            del bt
+            torch.cuda.empty_cache()
+
     head = cells.get((HEAD_MODE, HEAD_CTX)) or cells.get((HEAD_MODE, contexts[0])) or next(iter(cells.values()))
     head_ctx = head["context"]
     head_launches = head["launches_per_step"] * steps
@@ -412,6 +449,10 @@ def run_ours(args, rank, ws, local):
         "e2e": e2e,
         "modes": [cells[k] for k in sorted(cells, key=lambda k: (k[1], k[0]))],
         "crossings": crossing_report(bc, cfg, cells, contexts, sweep, sweep_ctx, sw_steps),
+        "batched": {"rows": batch_rows,
+                    "note": "bc_batch_step: B sequences, each with its own synthetic cache and tokens, decoding in "
+                            "lock step; the projections read the union of the batch's kept rows once, the LM head "
+                            "once; compared with B batch-1 steps of the same mode and context"},
     }
     if rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args, w, head_ctx)
@@ -966,6 +1007,9 @@ def main():
     ap.add_argument("--sweep-blocks", type=int, default=2,
                     help="blocks of the 2K-128K crossing sweep in 4K steps (0: no sweep)")
     ap.add_argument("--sweep-steps", type=int, default=8, help="timed steps per sweep cell (at most --steps)")
+    ap.add_argument("--batch-ctx", type=int, default=8192,
+                    help="context of the batched-step cells (one of --contexts; 0: none)")
+    ap.add_argument("--batches", type=int, nargs="+", default=[1, 2, 4, 8])
     ap.add_argument("--timeline", choices=("dense", "act", "kv", "both"),
                     help="per-site cost of one step in this mode at the first --contexts value")
     ap.add_argument("--record-traffic", metavar="NCU_RAW_CSV",

@@ -330,6 +330,59 @@ BC_API bc_status bc_attention(const float* q, const void* kv, int n_kv_heads, in
                               int Pmax, const int* pages, int n_pages, int n_tok,
                               float* out, void* scratch, size_t scratch_bytes, void* stream);
 
+/* ------------------------------------------------------------------ batched decode step */
+
+/* A batched decode step: `batch` sequences (1..8) share one model's weights
+ * and decode in lock step (ByteCross README, "Usage: The byte account":
+ * crossover_batch, where a batch reads the union of its sequences' kept
+ * projection weights once per step).  Each sequence has its own KV cache,
+ * page bounds, activations and selections, and all hold the same number of
+ * tokens.  Per layer every sequence keeps its own channels (its own top-k of
+ * |x| at every projection input, as at batch 1) and its own pages; each
+ * projection reads the union of the batch's kept rows once (the
+ * bc_gemv_batch kernels), the selections, page scores and attention run per
+ * sequence in batched grids, and the LM head reads its weights once for the
+ * whole batch.  Sequence b's result equals its batch-1 step up to fp32
+ * summation order.
+ *   kv_pools    device, batch * bc_kv_pool_bytes(cfg) bytes: sequence b's
+ *               pool starts at byte b * bc_kv_pool_bytes(cfg)
+ *   meta_pools  device, batch * bc_meta_pool_bytes(cfg) bytes, likewise
+ *   workspace   device, bc_batch_workspace_bytes(cfg, batch) bytes
+ * All three 256-byte aligned; the caller owns them and the stream.  cfg must
+ * also have a q/k/v width ((n_heads + 2 n_kv_heads) head_dim) that is a
+ * multiple of 128, and batch * hidden floats must fit one CTA's shared
+ * memory (the LM head holds every sequence's normed state: 227 KB on B200,
+ * so batch 8 up to hidden 7168).  Errors as for bc_model_create. */
+typedef struct bc_batch bc_batch;
+BC_API size_t bc_batch_workspace_bytes(const bc_config* cfg, int batch);
+BC_API bc_status bc_batch_create(const bc_config* cfg, const bc_weights* w, int batch, void* kv_pools,
+                                 void* meta_pools, void* workspace, size_t ws_bytes, void* stream,
+                                 bc_batch** out);
+BC_API bc_status bc_batch_destroy(bc_batch* b);
+/* CUDA graphs on (default) or off for later steps, as bc_set_graphs. */
+BC_API bc_status bc_batch_set_graphs(bc_batch* b, int enable);
+/* Tokens cached per sequence (the same for all). */
+BC_API int bc_batch_length(const bc_batch* b);
+/* Kernels launched since bc_batch_create. */
+BC_API long long bc_batch_launch_count(const bc_batch* b);
+/* Truncates every sequence's cache to n_ctx tokens, as bc_kv_reset. */
+BC_API bc_status bc_batch_reset(bc_batch* b, int n_ctx);
+/* Appends n_tokens keys and values to every sequence: k, v device bf16
+ * [batch][L][Hkv][n_tokens][hd], keys already rotated.  As bc_kv_append. */
+BC_API bc_status bc_batch_append(bc_batch* b, const void* k, const void* v, int n_tokens);
+/* One decode step of every sequence at position n = bc_batch_length(b):
+ * tokens host int [batch]; mode BC_DENSE, BC_ACT, BC_KV or BC_BOTH with rp,
+ * rkv, sinks, recent and page as for bc_decode_step; logits device f32
+ * [batch][vocab].  Async on the batch's stream; the length becomes n + 1.
+ * Errors: BC_EINVAL (bad mode, ratio, token), BC_ECAPACITY, BC_ECUDA. */
+BC_API bc_status bc_batch_step(bc_batch* b, const int* tokens, bc_mode mode, double rp, double rkv, int sinks,
+                               int recent, int page, float* logits);
+/* Per-sequence traces of the last batched step, as bc_trace, for sequence
+ * seq: BC_TRACE_XN, SEL_QKV, Q, ATTN, SEL_O, XN2, SEL_GU, H, SEL_D, X,
+ * PAGE_SCORES, PAGES and QKV (others: BC_EINVAL). */
+BC_API bc_status bc_batch_trace(const bc_batch* b, int seq, int layer, bc_trace_kind kind, const void** ptr,
+                                int* count, int* stride);
+
 /* ------------------------------------------------------------------ byte account */
 
 /* Bytes of one decode step.  Paper form: the pages' byte account (README,

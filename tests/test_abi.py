@@ -185,3 +185,25 @@ def test_library_keep_counts_where_float_ratios_round_up(n, mode, rp, rkv):
     if mode != "snap":
         P = -(-(n + 1) // 16)
         assert got["pages_kept"] == ba.page_keep(P, rkv, 1, 16)[0]
+
+
+def test_batch_entries_validate_on_host():
+    c = _cfg(TINY, 4096)
+    assert bc.bc_batch_workspace_bytes(C.byref(c), 0) == 0
+    assert bc.bc_batch_workspace_bytes(C.byref(c), 9) == 0
+    w1 = bc.bc_batch_workspace_bytes(C.byref(c), 1)
+    w4 = bc.bc_batch_workspace_bytes(C.byref(c), 4)
+    assert 0 < w1 < w4
+    bad = _cfg(dict(TINY, head_dim=96, hidden=768))
+    assert bc.bc_batch_workspace_bytes(C.byref(bad), 2) == 0
+    w = bc.bc_weights(*([C.c_void_p(256)] * 9))
+    h = C.c_void_p()
+    p = C.c_void_p(256)
+    assert bc.bc_batch_create(C.byref(c), C.byref(w), 9, p, p, p, 1 << 40, None, C.byref(h)) == bc.BC_EINVAL
+    assert bc.bc_batch_create(C.byref(c), C.byref(w), 2, None, p, p, 1 << 40, None, C.byref(h)) == bc.BC_EINVAL
+    assert bc.bc_batch_create(C.byref(c), C.byref(w), 2, p, p, p, 16, None, C.byref(h)) == bc.BC_ENOMEM
+    assert bc.bc_batch_create(C.byref(c), C.byref(w), 2, C.c_void_p(260), p, p, 1 << 40, None,
+                              C.byref(h)) == bc.BC_EINVAL
+    assert h.value is None
+    toks = (C.c_int * 2)(1, 2)
+    assert bc.bc_batch_step(None, toks, bc.BC_DENSE, 1.0, 1.0, 1, 16, 16, p) == bc.BC_EINVAL
