@@ -650,11 +650,12 @@ def cpu_threads():
 
 
 def cpu_baseline(args, w_dev, n_ctx):
-    """The oracle as it stands, on the host cores: layers 0-3 of one decode
-    step of the headline cell plus 1/32 of the LM head, scaled to a full step."""
+    """The oracle as it stands, on the host cores: layers 0-11 of one decode
+    step of the headline cell plus 1/32 of the LM head each (about 10 s of
+    CPU work), scaled to a full step."""
     from synth import LLAMA_8B
     cfg = LLAMA_8B
-    nl = 4
+    nl = 12
     wh, cache = host_sample_inputs(w_dev, n_ctx, nl)
     layer_s, head_s = [], 0.0
     for l in range(nl):
