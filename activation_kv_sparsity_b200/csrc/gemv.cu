@@ -21,7 +21,8 @@
 // fewer than 24 wide tiles) is shared by the CTAs of one or more thread-block
 // clusters, and the tile's k listed rows are cut into one contiguous run per
 // CTA.  A row segment is TW*2 bytes read by TW/8 lanes at 16 bytes each; a
-// CTA's 8 warps stream its run with 16 row segments per lane in flight;
+// CTA's 8 warps stream its run with 8 to 16 row segments per lane in flight
+// (two halves of 8 in registers, each refilled as soon as it is multiplied);
 // warps are reduced in shared memory.  The CTAs of a cluster then sum their partials
 // through distributed shared memory after a hardware cluster barrier (rank 0
 // reads them in rank order).  A tile split over several clusters adds one
@@ -207,27 +208,33 @@ __global__ void __launch_bounds__(kGemvThreads, 2) k_gemv(GemvArgs a) {
   float acc[8];
   #pragma unroll
   for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-  #pragma unroll
-  for (int u = 0; u < kRowsInFlight; ++u) {
-    const int rr = my0 + u * ROWS_STEP;
-    fma8(acc, rr < nr ? s_x[rr] : 0.f, w0[u]);
-  }
-  for (int r = my0 + ROWS_STEP * kRowsInFlight; r - lrow < nr; r += ROWS_STEP * kRowsInFlight) {
-    uint4 w[kRowsInFlight];
-    float xv[kRowsInFlight];
+  // Rolling pipeline over halves of 8 rows: w0[0..7] and w0[8..15] hold two
+  // halves; a half is refilled with the half two ahead as soon as it has been
+  // multiplied, so 8 to 16 rows per lane are always in flight.
+  constexpr int HALF = kRowsInFlight / 2;
+  const int rows_w = nr > warp * RPI ? (nr - warp * RPI + ROWS_STEP - 1) / ROWS_STEP : 0;
+  const int nh = (rows_w + HALF - 1) / HALF;
+  auto consume = [&](const uint4* w, int h) {
     #pragma unroll
-    for (int u = 0; u < kRowsInFlight; ++u) {
-      const int rr = r + u * ROWS_STEP;
-      if (rr < nr) {
-        w[u] = ld_stream(wcol + (size_t)s_idx[rr] * ld);
-        xv[u] = s_x[rr];
-      } else {
-        w[u] = make_uint4(0, 0, 0, 0);
-        xv[u] = 0.f;
-      }
+    for (int u = 0; u < HALF; ++u) {
+      const int rr = my0 + (h * HALF + u) * ROWS_STEP;
+      fma8(acc, rr < nr ? s_x[rr] : 0.f, w[u]);
     }
+  };
+  auto refill = [&](uint4* w, int h) {
     #pragma unroll
-    for (int u = 0; u < kRowsInFlight; ++u) fma8(acc, xv[u], w[u]);
+    for (int u = 0; u < HALF; ++u) {
+      const int rr = my0 + (h * HALF + u) * ROWS_STEP;
+      w[u] = rr < nr ? ld_stream(wcol + (size_t)s_idx[rr] * ld) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  for (int h = 0; h < nh; h += 2) {
+    consume(w0, h);
+    if (h + 2 < nh) refill(w0, h + 2);
+    if (h + 1 < nh) {
+      consume(w0 + HALF, h + 1);
+      if (h + 3 < nh) refill(w0 + HALF, h + 3);
+    }
   }
   // lanes of the same columns (different rows) first, then the warps
   #pragma unroll
