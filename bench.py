@@ -488,13 +488,20 @@ def crossing_report(bc, cfg, cells, contexts, sweep, sweep_ctx, sw_steps):
                "n_star_impl_tokens": impl_crossing(bc, cfg, rp, rkv)}
         if sweep:
             asc = sorted(sweep_ctx)
-            per_block = [crossing_of([(n, b[(ca, n)]["ms_per_step"] - b[(ck, n)]["ms_per_step"]) for n in asc])
-                         for b in sweep]
+            diffs = [[(n, b[(ca, n)]["ms_per_step"] - b[(ck, n)]["ms_per_step"]) for n in asc] for b in sweep]
+            per_block = [crossing_of(dd) for dd in diffs]
             row["measured_tokens_per_block"] = per_block
             found = [x for x in per_block if x is not None]
             row["measured_tokens"] = round(statistics.mean(found), 1) if found else None
             if found:
                 row["measured_range_tokens"] = [min(found), max(found)]
+            else:
+                # no sign change inside the sweep: say on which side the crossing lies
+                if all(dd[0][1] >= 0 for dd in diffs):
+                    row["measured_outside_sweep"] = f"below {asc[0]} tokens (kv already faster at the first context)"
+                elif all(dd[-1][1] < 0 for dd in diffs):
+                    row["measured_outside_sweep"] = f"above {asc[-1]} tokens (act still faster at the last context)"
+                row["diff_ms_first_last"] = [[round(dd[0][1], 4), round(dd[-1][1], 4)] for dd in diffs]
             if fit:
                 pred = predicted_crossing(bc, cfg, fit[0], fit[1], ca, ck)
                 row["cost_aware_predicted_tokens"] = pred
@@ -535,7 +542,7 @@ def cost_aware_fit(cells, contexts, kinds):
     when a cell is missing."""
     import numpy as np
     kinds = list(kinds)
-    if not all((m, n) in cells for m in kinds for n in contexts):
+    if len(contexts) < 2 or not all((m, n) in cells for m in kinds for n in contexts):
         return None
     rows, ys = [], []
     for j, m in enumerate(kinds):

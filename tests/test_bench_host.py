@@ -113,3 +113,19 @@ def test_sweep_fit_recovers_costs_and_predicts_every_pair():
             assert meas is None
             continue
         assert abs(meas - pred) <= 4096, (rp, rkv, meas, pred)
+
+
+def test_crossing_report_names_a_crossing_outside_the_sweep():
+    """When the kv branch is already faster at the sweep's first context the
+    report says the crossing lies below it instead of leaving it blank."""
+    ctx = [2048, 4096, 8192]
+    block = {}
+    for n in ctx:
+        block[("act@0.7", n)] = {"ms_per_step": 4.0, "bytes_per_step": 1e9}
+        block[("kv", n)] = {"ms_per_step": 3.9, "bytes_per_step": 1e9}
+        for c in ("dense", "act", "kv@0.5"):
+            block[(c, n)] = {"ms_per_step": 4.0, "bytes_per_step": 1e9}
+    rep = bench.crossing_report(bc, LLAMA_8B, {}, [], [block], ctx, 8)
+    row = rep["pairs"]["0.7/0.3"]
+    assert row["measured_tokens"] is None
+    assert row["measured_outside_sweep"].startswith("below 2048")
