@@ -335,6 +335,9 @@ extern "C" bc_status bc_kv_snap_select(bc_model* m, const float* q_obs, int n_ob
     BC_CUDA(launch_page_select(pa, m->stream, true), "snap page select");
   }
   m->launches += 4LL * L;
+  unsigned status = 0;
+  BC_CUDA(snap_status(&status, m->stream), "snap status");
+  if (status) return fail(BC_ECUDA, "snap scorer: a bounded wait gave up (status %u)", status);
   m->snap_valid = true;
   m->snap_P = P;
   m->snap_K = K;

@@ -109,7 +109,12 @@ struct SnapArgs {
   float* scores;                  // [Hkv][Pmax] page scores (attention mass)
 };
 int snap_chunks(int n_tok);
+// head_dim 128 with at most 64 observation queries per kv head runs on the
+// tcgen05 tensor cores, other shapes on mma.sync
 cudaError_t launch_snap_scores(const SnapArgs& a, cudaStream_t st, bool pdl);
+// Synchronises the stream and reads the tcgen05 scorer's status word: 0, or
+// the bits of the waits that gave up (a lost copy or MMA completion).
+cudaError_t snap_status(unsigned* status, cudaStream_t st);
 
 // ------------------------------------------------------------------ attention
 struct AttnArgs {

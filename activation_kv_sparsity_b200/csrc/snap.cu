@@ -27,7 +27,10 @@
 // per decode step.
 #include "common.cuh"
 #include "kernels.h"
+#include "tensor_map.h"
 
+#include <math.h>
+#include <string.h>
 #include <algorithm>
 
 namespace bc {
@@ -217,6 +220,401 @@ __global__ void k_snap_merge(SnapArgs a, int chunks) {
 
 int snap_chunks(int n_tok) { return (n_tok + kSnapTok - 1) / kSnapTok; }
 
+// ------------------------------------------------------------------ tcgen05 scorer
+// The same two passes for head_dim 128 and at most 64 observation queries per
+// kv head, with the logits of a tile of 256 keys (16 pages) computed on the
+// fifth-generation tensor cores into tensor memory.
+//
+// Operands.  A (shared memory, 128 rows x 128 dims bf16, K-major, 128-byte
+// swizzle, written by the CTA): row 2q holds the bf16 "hi" part of
+// observation query q scaled by log2(e)/sqrt(hd), row 2q+1 its residue, so
+// D[2q] + D[2q+1] is the base-2 logit with about 16 bits of the fp32 query.
+// B (shared memory, 256 keys x 128 dims): two tensor copies of 64 dims each
+// through a 3-D tensor map over [page][token][dim] whose page stride skips
+// the values.  D: 128 lanes x 256 fp32 columns of tensor memory; two such
+// accumulators, so one tile's epilogue runs while the next is multiplied.
+//
+// Roles (18 warps): warp 0 issues the tensor copies into a 2-stage ring of
+// 64 KB; warp 1 owns the tensor memory, and one of its threads issues the
+// MMAs (8 per tile: two 64-dim halves x four k16 steps, M 128, N 256) and
+// commits them to the stage's and the accumulator's mbarriers; warps 2-17
+// read the accumulator, each a 32-lane subpartition (its warp index mod 4,
+// as tensor memory requires) and a group of 64 columns (4 pages).  A lane
+// holds one row, so lanes 2q and 2q+1 hold query q; they swap half their
+// columns so that each ends with the 16 logits of one page.  Sixteen reading
+// warps keep the exponentials and shuffles of a tile within the time its
+// keys take to arrive.  A chunk's tiles are split evenly over the CTAs of a
+// kv head, one CTA per SM.  Every wait is bounded; a
+// timeout sets g_snap_status (read by the host after the selection) and the
+// CTA still releases its tensor memory after its own copies and MMAs.
+constexpr int kTcKeys = 256;                          // keys per tile
+constexpr int kTcPagesPerTile = kTcKeys / kPage;      // 16
+constexpr int kTcHalfBytes = kTcKeys * 128;           // 64 dims of a tile: 32 KB
+constexpr int kTcStageBytes = 2 * kTcHalfBytes;       // 64 KB
+constexpr int kTcStages = 2;
+constexpr int kTcABytes = 2 * 128 * 128;              // two 64-dim halves of 128 rows
+constexpr int kTcSmem = 1024 + kTcABytes + kTcStages * kTcStageBytes;
+constexpr int kTcEpiWarps = 16;                       // 4 subpartitions x 4 column groups
+constexpr int kTcColGroup = kTcKeys / (kTcEpiWarps / 4);   // 64 columns
+constexpr int kTcThreads = (2 + kTcEpiWarps) * 32;
+constexpr uint32_t kTcCols = 512;                     // two 256-column accumulators
+// instruction descriptor: fp32 D, bf16 A and B, both K-major, N 256, M 128
+constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTcKeys >> 3) << 17) |
+                              ((uint32_t)(128 >> 4) << 24);
+
+__device__ unsigned g_snap_status;
+
+struct SnapTcParams {
+  CUtensorMap tm;          // keys of the layer: [Hkv*Pmax pages][16 tokens][128 dims], box 64 x 16 x 16
+  SnapArgs a;
+  int chunks;              // CTAs per kv head; chunk c takes tiles [c*T/chunks, (c+1)*T/chunks)
+};
+
+// Shared-memory matrix descriptor: K-major rows of 128 bytes, 128-byte
+// swizzle, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t tc_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(kTcIdesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_load_tile(uint32_t dst, const void* tmap, int d0, int page, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(tmap), "r"(d0), "r"(0), "r"(page), "r"(bar)
+      : "memory");
+}
+// 32 consecutive fp32 columns of this warp's 32 lanes (complete after
+// tcgen05.wait::ld).
+__device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+
+template <int PASS>
+__global__ void __launch_bounds__(kTcThreads, 1) k_snap_tc(const __grid_constant__ SnapTcParams prm) {
+  const SnapArgs& a = prm.a;
+  extern __shared__ __align__(1024) unsigned char tc_smem[];
+  __shared__ __align__(8) uint64_t full_b[kTcStages], empty_b[kTcStages], acc_full[2], acc_empty[2];
+  __shared__ uint32_t s_taddr;
+  __shared__ int s_err;
+  __shared__ float s_wm[4][kTcPagesPerTile];          // PASS 1: [subpartition][page of the tile]
+  __shared__ float2 s_ml[4][128];                     // PASS 0: [column group][row] (max, sum)
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int chunk = blockIdx.x, h = blockIdx.y;
+  const int Q = a.n_obs * a.G;
+  const int P = (a.n_tok + kPage - 1) / kPage;
+  const int T = (P + kTcPagesPerTile - 1) / kTcPagesPerTile;
+  const int t0 = (int)((long long)chunk * T / prm.chunks);
+  const int nt = (int)((long long)(chunk + 1) * T / prm.chunks) - t0;
+  const uint32_t s0 = smem_addr(tc_smem);
+  const uint32_t sA = (s0 + 1023u) & ~1023u, sB = sA + kTcABytes;
+  unsigned char* gA = tc_smem + (sA - s0);
+
+  if (tid == 0) {
+    for (int i = 0; i < kTcStages; ++i) {
+      mbar_init(smem_addr(&full_b[i]), 1);
+      mbar_init(smem_addr(&empty_b[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_addr(&acc_full[i]), 1);
+      mbar_init(smem_addr(&acc_empty[i]), kTcEpiWarps);
+    }
+    mbar_init_fence();
+    s_err = 0;
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_taddr)),
+                 "r"(kTcCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  // the keys do not depend on the previous kernel: the first tiles' copies
+  // start before waiting for it and before A is built (barrier init is
+  // ordered by the same thread)
+  auto issue = [&](int it) {
+    const int st = it & 1;
+    const uint32_t fb = smem_addr(&full_b[st]);
+    mbar_arrive_expect_tx(fb, kTcStageBytes);
+    const int page = h * a.Pmax + (t0 + it) * kTcPagesPerTile;
+    tc_load_tile(sB + st * kTcStageBytes, &prm.tm, 0, page, fb);
+    tc_load_tile(sB + st * kTcStageBytes + kTcHalfBytes, &prm.tm, 64, page, fb);
+  };
+  const int pre = min(nt, kTcStages);
+  if (tid == 0)
+    for (int it = 0; it < pre; ++it) issue(it);
+  pdl_wait();
+  pdl_trigger();
+
+  // A: row r = 2q + (0 hi | 1 lo), 16-byte chunk c of dims 8c .. 8c+7 (half
+  // c / 8), stored at chunk (c % 8) ^ (r % 8) of the row: the 128-byte swizzle
+  const float qscale = 1.4426950408889634f * rsqrtf(128.f);
+  for (int e = tid; e < 128 * 16; e += kTcThreads) {
+    const int row = e >> 4, c = e & 15, q = row >> 1;
+    float v[8];
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    if (q < Q) {
+      const int j = q / a.G, gg = q % a.G;
+      const float4* qp = reinterpret_cast<const float4*>(a.q_obs + ((size_t)j * a.Hkv * a.G + h * a.G + gg) * 128 + c * 8);
+      const float4 x0 = qp[0], x1 = qp[1];
+      v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+      v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+    }
+    uint32_t w[4];
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t hi, lo;
+      split2(v[2 * i] * qscale, v[2 * i + 1] * qscale, hi, lo);
+      w[i] = (row & 1) ? lo : hi;
+    }
+    const uint32_t off = (c >> 3) * (128 * 128) + row * 128 + (((c & 7) ^ (row & 7)) << 4);
+    *reinterpret_cast<uint4*>(gA + off) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // A is read by the tensor cores
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_taddr;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = pre;
+      for (int it = pre; it < nt; ++it) {
+        if (!mbar_wait(smem_addr(&empty_b[it & 1]), ((it >> 1) - 1) & 1)) {
+          atomicOr(&g_snap_status, 1u);
+          break;
+        }
+        issue(it);
+        issued = it + 1;
+      }
+      // the last copies have landed before the CTA ends (they have, unless a
+      // wait above gave up)
+      for (int it = max(0, issued - kTcStages); it < issued; ++it)
+        mbar_wait(smem_addr(&full_b[it & 1]), (it >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < nt; ++it) {
+        const int st = it & 1;
+        if (!mbar_wait(smem_addr(&full_b[st]), (it >> 1) & 1) ||
+            (it >= 2 && !mbar_wait(smem_addr(&acc_empty[st]), ((it >> 1) - 1) & 1))) {
+          atomicOr(&g_snap_status, 2u);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + st * kTcKeys;
+        #pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          #pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            tc_mma(d, tc_desc(sA + hh * (128 * 128) + ks * 32),
+                   tc_desc(sB + st * kTcStageBytes + hh * kTcHalfBytes + ks * 32), (hh | ks) != 0);
+        tc_commit(smem_addr(&empty_b[st]));
+        tc_commit(smem_addr(&acc_full[st]));
+        issued = it + 1;
+      }
+      // every MMA issued has completed before the tensor memory is released
+      if (issued > 0) mbar_wait(smem_addr(&acc_full[(issued - 1) & 1]), ((issued - 1) >> 1) & 1);
+    }
+  } else {
+    const int ew = warp - 2, sp = warp & 3;          // tensor-memory subpartition: lanes 32*sp ..
+    const int cg = ew >> 2;                          // column group: columns 64*cg .. 64*cg + 63
+    const int q = (32 * sp + lane) >> 1;
+    const bool odd = lane & 1, qv = q < Q;
+    float m_run = -INFINITY, l_run = 0.f, M = 0.f, invL = 0.f;
+    if (PASS == 1 && qv) {
+      const float2 st = a.stats[(size_t)h * Q + q];
+      M = st.x;
+      invL = 1.0f / st.y;
+    }
+    for (int it = 0; it < nt; ++it) {
+      const int st = it & 1;
+      bool ok = *reinterpret_cast<volatile int*>(&s_err) == 0;
+      if (ok && !mbar_wait(smem_addr(&acc_full[st]), (it >> 1) & 1)) {
+        ok = false;
+        s_err = 1;
+        atomicOr(&g_snap_status, 4u);
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+      const int key_t = (t0 + it) * kTcKeys + cg * kTcColGroup;
+      if (ok) {
+        // this warp's 64 columns: two loads in flight, one wait
+        uint32_t v[2][32];
+        const uint32_t ta = tmem + ((uint32_t)(32 * sp) << 16) + st * kTcKeys + cg * kTcColGroup;
+        tc_ld32_nowait(ta, v[0]);
+        tc_ld32_nowait(ta + 32, v[1]);
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        #pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          // lanes 2q (hi) and 2q+1 (lo): the even lane keeps columns 0-15, the odd one 16-31
+          float lg[16];
+          #pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const uint32_t send = odd ? v[c][j] : v[c][16 + j];
+            const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 1);
+            lg[j] = __uint_as_float(odd ? v[c][16 + j] : v[c][j]) + __uint_as_float(recv);
+          }
+          const int key0 = key_t + c * 32 + (odd ? 16 : 0);
+          const int valid = qv ? min(kPage, max(0, a.n_tok - key0)) : 0;
+          if (PASS == 0) {
+            if (valid > 0) {
+              float mx = -INFINITY;
+              #pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (j < valid) mx = fmaxf(mx, lg[j]);
+              const float m_new = fmaxf(m_run, mx);
+              float add = 0.f;
+              #pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (j < valid) add += exp2f(lg[j] - m_new);
+              l_run = (m_run == -INFINITY ? 0.f : l_run * exp2f(m_run - m_new)) + add;
+              m_run = m_new;
+            }
+          } else {
+            float mass = 0.f;
+            #pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (j < valid) mass += exp2f(lg[j] - M) * invL;
+            // the warp's 16 queries of this page: lanes of the same parity
+            #pragma unroll
+            for (int o = 2; o < 32; o <<= 1) mass += __shfl_xor_sync(0xffffffffu, mass, o);
+            if (lane < 2) s_wm[sp][cg * 4 + c * 2 + lane] = mass;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&acc_empty[st]));
+      if (PASS == 1) {
+        // the tile's page masses: the four subpartitions' sums, in order
+        asm volatile("bar.sync 1, %0;" ::"n"(kTcEpiWarps * 32) : "memory");
+        if (ew == 0 && lane < kTcPagesPerTile && ok) {
+          const int page = (t0 + it) * kTcPagesPerTile + lane;
+          if (page < P)
+            a.scores[(size_t)h * a.Pmax + page] = ((s_wm[0][lane] + s_wm[1][lane]) + s_wm[2][lane]) + s_wm[3][lane];
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kTcEpiWarps * 32) : "memory");
+      }
+    }
+    if (PASS == 0) {
+      // the pair's two halves of each page, then the four column groups in order
+      const float m2 = __shfl_xor_sync(0xffffffffu, m_run, 1), l2 = __shfl_xor_sync(0xffffffffu, l_run, 1);
+      const float mm = fmaxf(m_run, m2);
+      const float l = mm == -INFINITY ? 0.f
+                                      : (m_run == -INFINITY ? 0.f : l_run * exp2f(m_run - mm)) +
+                                            (m2 == -INFINITY ? 0.f : l2 * exp2f(m2 - mm));
+      s_ml[cg][32 * sp + lane] = make_float2(mm, l);
+      asm volatile("bar.sync 1, %0;" ::"n"(kTcEpiWarps * 32) : "memory");
+      if (cg == 0 && !odd && qv) {
+        float M2 = -INFINITY;
+        #pragma unroll
+        for (int g = 0; g < 4; ++g) M2 = fmaxf(M2, s_ml[g][32 * sp + lane].x);
+        float L2 = 0.f;
+        #pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float2 p = s_ml[g][32 * sp + lane];
+          if (p.x != -INFINITY) L2 += p.y * exp2f(p.x - M2);
+        }
+        a.part[((size_t)h * gridDim.x + chunk) * Q + q] = make_float2(M2, L2);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcCols) : "memory");
+  }
+}
+
+static int device_sms() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 1;
+  }
+  return sms;
+}
+
+static cudaError_t launch_tc(const SnapArgs& a, cudaStream_t st, bool pdl) {
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(k_snap_tc<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_snap_tc<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const EncodeTiledFn encode = tensor_map_encoder();
+  if (!encode) return cudaErrorNotSupported;
+  SnapTcParams prm;
+  memset(&prm, 0, sizeof prm);
+  prm.a = a;
+  // the layer's keys as [Hkv*Pmax pages][16 tokens][128 dims]: the page
+  // stride (keys and values of a page) skips the values
+  cuuint64_t gdim[3] = {128, (cuuint64_t)kPage, (cuuint64_t)a.Hkv * a.Pmax};
+  cuuint64_t gstride[2] = {128 * sizeof(__nv_bfloat16), 2 * kPage * 128 * sizeof(__nv_bfloat16)};
+  cuuint32_t box[3] = {64, (cuuint32_t)kPage, (cuuint32_t)kTcPagesPerTile};
+  cuuint32_t estride[3] = {1, 1, 1};
+  if ((uintptr_t)a.kv & 15) return cudaErrorInvalidValue;
+  if (encode(&prm.tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void*)a.kv, gdim, gstride, box, estride,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  // one CTA per SM at most: chunks of whole tiles, no more chunks than the
+  // (max, sum) buffer holds
+  const int P = (a.n_tok + kPage - 1) / kPage;
+  const int T = (P + kTcPagesPerTile - 1) / kTcPagesPerTile;
+  int chunks = std::min(T, std::min(std::max(1, device_sms() / a.Hkv), snap_chunks(a.n_tok)));
+  prm.chunks = chunks;
+  const int Q = a.n_obs * a.G;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(chunks, a.Hkv);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = kTcSmem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_snap_tc<0>, prm);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t c2 = cfg;
+  c2.gridDim = dim3((a.Hkv * Q + 127) / 128);
+  c2.blockDim = dim3(128);
+  c2.dynamicSmemBytes = 0;
+  e = cudaLaunchKernelEx(&c2, k_snap_merge, a, chunks);
+  if (e != cudaSuccess) return e;
+  return cudaLaunchKernelEx(&cfg, k_snap_tc<1>, prm);
+}
+
+cudaError_t snap_status(unsigned* status, cudaStream_t st) {
+  cudaError_t e = cudaMemcpyFromSymbolAsync(status, g_snap_status, sizeof(unsigned), 0, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  return e;
+}
+
 template <int HD>
 static cudaError_t launch_hd(const SnapArgs& a, cudaStream_t st, bool pdl) {
   constexpr int KSTEPS = HD / 16;
@@ -256,6 +654,7 @@ static cudaError_t launch_hd(const SnapArgs& a, cudaStream_t st, bool pdl) {
 
 cudaError_t launch_snap_scores(const SnapArgs& a, cudaStream_t st, bool pdl) {
   if (a.n_tok < 1 || a.n_obs < 1 || a.n_obs * a.G > kSnapMaxQ) return cudaErrorInvalidValue;
+  if (a.hd == 128 && a.n_obs * a.G <= 64) return launch_tc(a, st, pdl);
   if (a.hd == 128) return launch_hd<128>(a, st, pdl);
   if (a.hd == 64) return launch_hd<64>(a, st, pdl);
   return cudaErrorInvalidValue;

@@ -786,16 +786,34 @@ def run_kernel_only(args, local):
         for _ in range(args.warmup):
             launch()
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(model.stream)
-        for _ in range(args.steps):
-            launch()
-        e1.record(model.stream)
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / args.steps
+        # the selection ends by reading the scorer's status word (a host
+        # sync), so it is timed on the device: CUPTI kernel timestamps, from
+        # a selection's first kernel's start to its last kernel's end
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            for _ in range(args.steps):
+                launch()
+            torch.cuda.synchronize()
+        ev = sorted((e for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA
+                     and e.name.split("(")[0].split("<")[0].split("::")[-1] in
+                     ("k_snap", "k_snap_tc", "k_snap_merge", "k_page_select", "k_page_select_cta")),
+                    key=lambda e: e.time_range.start)
+        per = 4 * c2["n_layers"]
+        if len(ev) != per * args.steps:
+            return {"kernel": "snap", "error": f"{len(ev)} kernels traced, expected {per * args.steps}"}
+        spans = [ev[i * per + per - 1].time_range.end - ev[i * per].time_range.start for i in range(args.steps)]
+        kern = {}
+        for e in ev:
+            nm = e.name.split("(")[0]
+            kern.setdefault(nm, []).append(e.time_range.end - e.time_range.start)
+        ms = sum(spans) / len(spans) / 1000.0
+        keys = 2 * c2["n_layers"] * c2["n_kv_heads"] * n * c2["head_dim"] * 2     # key bytes read, both passes
         return {"kernel": "snap", "ms_per_selection": round(ms, 4), "flops": flops,
-                "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
-                "note": "2 layers at 32K, both passes and the page select; mma.sync m16n8k16, bf16 keys, hi/lo-split queries"}
+                "tflops": round(flops / (ms * 1e-3) / 1e12, 2), "key_bytes": keys,
+                "key_gbs": round(keys / (ms * 1e-3) / 1e9, 1),
+                "us_per_kernel": {k: round(sum(v) / len(v), 2) for k, v in kern.items()},
+                "note": "2 layers at 32K, both passes, the merge and the page select, device span per selection "
+                        "(CUPTI); tcgen05 M128 N256 K16, keys by tensor copies, hi/lo-split queries"}
     if args.only_kernel == "gemv_batch":
         return run_batch_gemv(args, dev, stream, cfg)
     if args.only_kernel in ("gemv_gateup", "gemv_gateup_dense"):

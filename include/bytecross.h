@@ -169,8 +169,13 @@ BC_API bc_status bc_kv_append(bc_model* m, const void* k, const void* v, int n_t
  *   n_obs  1 <= n_obs and n_obs*G <= 128.
  * Runs four kernels per layer on the model's stream (not captured in the
  * step graphs); the selection is voided by bc_kv_append and bc_kv_reset.
+ * With hd = 128 and n_obs*G <= 64 the logits run on the tcgen05 tensor
+ * cores (tensor-memory accumulators, keys brought by tensor copies), other
+ * shapes on mma.sync.  Returns after the stream has drained, having read
+ * the scorer's status word (its bounded waits).
  * Traces: BC_TRACE_SNAP_SCORES, BC_TRACE_SNAP_PAGES.
- * Errors: BC_EINVAL (no tokens, bad sizes or ratios), BC_ECUDA. */
+ * Errors: BC_EINVAL (no tokens, bad sizes or ratios), BC_ECUDA (also when a
+ * bounded wait of the scorer gave up). */
 BC_API bc_status bc_kv_snap_select(bc_model* m, const float* q_obs, int n_obs, double rkv, int sinks,
                                    int recent);
 

@@ -155,3 +155,29 @@ def test_llama8b_shape_snap_scores():
     cache.extend(bits(k), bits(v))
     _check_selection(cfg, cache, q_obs.cpu(), scores, pages, 16)
     m.close()
+
+
+@pytest.mark.parametrize("n,n_obs", [(4096 + 16 * 37 + 5, 16), (40000 + 3, 16), (2560 + 7, 3), (3000, 32)])
+def test_llama8b_shape_snap_tensor_core_path(n, n_obs):
+    """The 8B layer shape (two layers) against the oracle where the scorer
+    runs on tcgen05 (head_dim 128, n_obs*G <= 64): a ragged last page and
+    tile, chunks of many tiles (40K tokens: both ring stages and both
+    accumulators reused), few queries (12 of the 64 rows); and one shape
+    beyond 64 queries, which stays on the mma.sync scorer."""
+    cfg = dict(LLAMA_8B, n_layers=2)
+    w = make_weights(cfg, seed=0, device=DEV)
+    k, v = make_kv(cfg, n, seed=1, device=DEV)
+    m = bc.Model(cfg, w, n + 16)
+    m.append(k, v)
+    q_obs = obs_queries(cfg, n_obs, seed=11, device=DEV)
+    m.snap_select(q_obs, **SEL)
+    torch.cuda.synchronize()
+    scores, pages = _snap_traces(m, cfg)
+    cache = od.Cache(cfg, n + 16)
+    cache.extend(bits(k), bits(v))
+    _check_selection(cfg, cache, q_obs.cpu(), scores, pages, n_obs)
+    P = (n + 15) // 16
+    G = cfg["n_heads"] // cfg["n_kv_heads"]
+    for sc in scores.values():
+        assert sc.shape == (P,) and abs(sc.sum() - n_obs * G) < 1e-3 * n_obs * G
+    m.close()
