@@ -81,6 +81,7 @@ struct Layout {
   size_t pscore, pages;                                         // [L][Hkv][Pmax]
   size_t snap_scores, snap_pages;                               // [L][Hkv][Pmax]
   size_t snap_part, snap_stats;                                 // float2 [Hkv][chunks][Q], [Hkv][Q]
+  size_t snap_pp;                                               // float2 [Hkv][Pmax][64] (one layer)
   size_t part_o, part_ml, gemv_part, counters;
   size_t total;
   int nqkv, hq, Pmax, max_dout;
@@ -124,6 +125,7 @@ static Layout make_layout(const bc_config* c) {
   y.snap_pages = take(4 * L * c->n_kv_heads * (size_t)y.Pmax);
   y.snap_part = take(8 * (size_t)c->n_kv_heads * snap_chunks(c->max_ctx) * kSnapMaxQ);
   y.snap_stats = take(8 * (size_t)c->n_kv_heads * kSnapMaxQ);
+  y.snap_pp = c->head_dim == 128 ? take(8 * (size_t)c->n_kv_heads * y.Pmax * 64) : o;
   y.part_o = take(4 * (size_t)c->n_heads * kMaxSplits * c->head_dim);
   y.part_ml = take(4 * (size_t)c->n_heads * kMaxSplits * 2);
   y.gemv_part = take(4 * (size_t)kGemvMaxContrib * y.max_dout);
@@ -329,6 +331,7 @@ extern "C" bc_status bc_kv_snap_select(bc_model* m, const float* q_obs, int n_ob
     sa.part = at<float2>(m, y.snap_part);
     sa.stats = at<float2>(m, y.snap_stats);
     sa.scores = at<float>(m, y.snap_scores) + (size_t)l * Hkv * Pmax;
+    sa.pp = c.head_dim == 128 ? at<float2>(m, y.snap_pp) : nullptr;
     BC_CUDA(launch_snap_scores(sa, m->stream, true), "snap page scores");
     PageArgs pa{nullptr, nullptr, Hkv, G, c.head_dim, Pmax, P, K, sinks, recent, 0, sa.scores,
                 at<int>(m, y.snap_pages) + (size_t)l * Hkv * Pmax, nullptr};

@@ -107,10 +107,12 @@ struct SnapArgs {
   float2* part;                   // [Hkv][snap_chunks(n_tok)][Q] per-chunk (max, sum), base 2
   float2* stats;                  // [Hkv][Q] (max, sum) over all n_tok tokens
   float* scores;                  // [Hkv][Pmax] page scores (attention mass)
+  float2* pp;                     // tcgen05 scorer: [Hkv][Pmax][Q] each page's (max, sum) per query
 };
 int snap_chunks(int n_tok);
-// head_dim 128 with at most 64 observation queries per kv head runs on the
-// tcgen05 tensor cores, other shapes on mma.sync
+// head_dim 128 with at most 64 observation queries per kv head (and pp set)
+// runs in one pass over the keys on the tcgen05 tensor cores, other shapes in
+// two passes on mma.sync
 cudaError_t launch_snap_scores(const SnapArgs& a, cudaStream_t st, bool pdl);
 // Synchronises the stream and reads the tcgen05 scorer's status word: 0, or
 // the bits of the waits that gave up (a lost copy or MMA completion).

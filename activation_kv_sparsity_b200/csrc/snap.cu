@@ -221,9 +221,17 @@ __global__ void k_snap_merge(SnapArgs a, int chunks) {
 int snap_chunks(int n_tok) { return (n_tok + kSnapTok - 1) / kSnapTok; }
 
 // ------------------------------------------------------------------ tcgen05 scorer
-// The same two passes for head_dim 128 and at most 64 observation queries per
-// kv head, with the logits of a tile of 256 keys (16 pages) computed on the
-// fifth-generation tensor cores into tensor memory.
+// For head_dim 128 and at most 64 observation queries per kv head: one pass
+// over the keys, with the logits of a tile of 256 keys (16 pages) computed on
+// the fifth-generation tensor cores into tensor memory.  For every page and
+// query it keeps the page's own (max m_pq, sum l_pq) of exp2(s - m_pq), and
+// per chunk of pages the running (max, sum) of every query; after the merge
+// of the chunks (M_q, L_q), a small kernel forms each page's mass
+//
+//   score_p = sum_q l_pq * exp2(m_pq - M_q) / L_q,
+//
+// the same sum as above regrouped by page, so the keys are read once (the
+// page partials add 512 bytes per page, an eighth of the page's keys).
 //
 // Operands.  A (shared memory, 128 rows x 128 dims bf16, K-major, 128-byte
 // swizzle, written by the CTA): row 2q holds the bf16 "hi" part of
@@ -308,15 +316,13 @@ __device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t (&v)[32]
       : "r"(taddr));
 }
 
-template <int PASS>
 __global__ void __launch_bounds__(kTcThreads, 1) k_snap_tc(const __grid_constant__ SnapTcParams prm) {
   const SnapArgs& a = prm.a;
   extern __shared__ __align__(1024) unsigned char tc_smem[];
   __shared__ __align__(8) uint64_t full_b[kTcStages], empty_b[kTcStages], acc_full[2], acc_empty[2];
   __shared__ uint32_t s_taddr;
   __shared__ int s_err;
-  __shared__ float s_wm[4][kTcPagesPerTile];          // PASS 1: [subpartition][page of the tile]
-  __shared__ float2 s_ml[4][128];                     // PASS 0: [column group][row] (max, sum)
+  __shared__ float2 s_ml[4][128];                     // [column group][row] (max, sum)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int chunk = blockIdx.x, h = blockIdx.y;
   const int Q = a.n_obs * a.G;
@@ -440,12 +446,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_snap_tc(const __grid_constant
     const int cg = ew >> 2;                          // column group: columns 64*cg .. 64*cg + 63
     const int q = (32 * sp + lane) >> 1;
     const bool odd = lane & 1, qv = q < Q;
-    float m_run = -INFINITY, l_run = 0.f, M = 0.f, invL = 0.f;
-    if (PASS == 1 && qv) {
-      const float2 st = a.stats[(size_t)h * Q + q];
-      M = st.x;
-      invL = 1.0f / st.y;
-    }
+    float m_run = -INFINITY, l_run = 0.f;
     for (int it = 0; it < nt; ++it) {
       const int st = it & 1;
       bool ok = *reinterpret_cast<volatile int*>(&s_err) == 0;
@@ -476,47 +477,28 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_snap_tc(const __grid_constant
           }
           const int key0 = key_t + c * 32 + (odd ? 16 : 0);
           const int valid = qv ? min(kPage, max(0, a.n_tok - key0)) : 0;
-          if (PASS == 0) {
-            if (valid > 0) {
-              float mx = -INFINITY;
-              #pragma unroll
-              for (int j = 0; j < 16; ++j)
-                if (j < valid) mx = fmaxf(mx, lg[j]);
-              const float m_new = fmaxf(m_run, mx);
-              float add = 0.f;
-              #pragma unroll
-              for (int j = 0; j < 16; ++j)
-                if (j < valid) add += exp2f(lg[j] - m_new);
-              l_run = (m_run == -INFINITY ? 0.f : l_run * exp2f(m_run - m_new)) + add;
-              m_run = m_new;
-            }
-          } else {
-            float mass = 0.f;
+          if (valid > 0) {
+            // this page's (max, sum) for query q, then the running pair
+            float mp = -INFINITY;
             #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (j < valid) mass += exp2f(lg[j] - M) * invL;
-            // the warp's 16 queries of this page: lanes of the same parity
+              if (j < valid) mp = fmaxf(mp, lg[j]);
+            float lp = 0.f;
             #pragma unroll
-            for (int o = 2; o < 32; o <<= 1) mass += __shfl_xor_sync(0xffffffffu, mass, o);
-            if (lane < 2) s_wm[sp][cg * 4 + c * 2 + lane] = mass;
+            for (int j = 0; j < 16; ++j)
+              if (j < valid) lp += exp2f(lg[j] - mp);
+            a.pp[((size_t)h * a.Pmax + key0 / kPage) * Q + q] = make_float2(mp, lp);
+            const float m_new = fmaxf(m_run, mp);
+            l_run = (m_run == -INFINITY ? 0.f : l_run * exp2f(m_run - m_new)) + lp * exp2f(mp - m_new);
+            m_run = m_new;
           }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(&acc_empty[st]));
-      if (PASS == 1) {
-        // the tile's page masses: the four subpartitions' sums, in order
-        asm volatile("bar.sync 1, %0;" ::"n"(kTcEpiWarps * 32) : "memory");
-        if (ew == 0 && lane < kTcPagesPerTile && ok) {
-          const int page = (t0 + it) * kTcPagesPerTile + lane;
-          if (page < P)
-            a.scores[(size_t)h * a.Pmax + page] = ((s_wm[0][lane] + s_wm[1][lane]) + s_wm[2][lane]) + s_wm[3][lane];
-        }
-        asm volatile("bar.sync 1, %0;" ::"n"(kTcEpiWarps * 32) : "memory");
-      }
     }
-    if (PASS == 0) {
+    {
       // the pair's two halves of each page, then the four column groups in order
       const float m2 = __shfl_xor_sync(0xffffffffu, m_run, 1), l2 = __shfl_xor_sync(0xffffffffu, l_run, 1);
       const float mm = fmaxf(m_run, m2);
@@ -547,6 +529,46 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_snap_tc(const __grid_constant
   }
 }
 
+// Page masses from the page partials: a warp per page, lane l holding
+// queries l and l + 32; the butterfly sum fixes the order.
+constexpr int kMassWarps = 8;
+constexpr int kMassPagesPerBlock = 64;
+
+__global__ void __launch_bounds__(kMassWarps * 32) k_snap_mass(SnapArgs a) {
+  const int h = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int Q = a.n_obs * a.G, P = (a.n_tok + kPage - 1) / kPage;
+  pdl_wait();
+  pdl_trigger();
+  float M[2], invL[2];
+  #pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int q = lane + 32 * u;
+    M[u] = 0.f;
+    invL[u] = 0.f;
+    if (q < Q) {
+      const float2 st = a.stats[(size_t)h * Q + q];
+      M[u] = st.x;
+      invL[u] = 1.0f / st.y;
+    }
+  }
+  const int p_end = min(P, (blockIdx.x + 1) * kMassPagesPerBlock);
+  for (int page = blockIdx.x * kMassPagesPerBlock + warp; page < p_end; page += kMassWarps) {
+    const float2* pp = a.pp + ((size_t)h * a.Pmax + page) * Q;
+    float mass = 0.f;
+    #pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int q = lane + 32 * u;
+      if (q < Q) {
+        const float2 v = pp[q];
+        mass += v.y * exp2f(v.x - M[u]) * invL[u];
+      }
+    }
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mass += __shfl_xor_sync(0xffffffffu, mass, o);
+    if (lane == 0) a.scores[(size_t)h * a.Pmax + page] = mass;
+  }
+}
+
 static int device_sms() {
   static int sms = 0;
   if (!sms) {
@@ -560,8 +582,7 @@ static int device_sms() {
 static cudaError_t launch_tc(const SnapArgs& a, cudaStream_t st, bool pdl) {
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(k_snap_tc<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_snap_tc<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem);
+    cudaError_t e = cudaFuncSetAttribute(k_snap_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmem);
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
@@ -598,7 +619,7 @@ static cudaError_t launch_tc(const SnapArgs& a, cudaStream_t st, bool pdl) {
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, k_snap_tc<0>, prm);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, k_snap_tc, prm);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t c2 = cfg;
   c2.gridDim = dim3((a.Hkv * Q + 127) / 128);
@@ -606,7 +627,10 @@ static cudaError_t launch_tc(const SnapArgs& a, cudaStream_t st, bool pdl) {
   c2.dynamicSmemBytes = 0;
   e = cudaLaunchKernelEx(&c2, k_snap_merge, a, chunks);
   if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&cfg, k_snap_tc<1>, prm);
+  cudaLaunchConfig_t c3 = c2;
+  c3.gridDim = dim3((P + kMassPagesPerBlock - 1) / kMassPagesPerBlock, a.Hkv);
+  c3.blockDim = dim3(kMassWarps * 32);
+  return cudaLaunchKernelEx(&c3, k_snap_mass, a);
 }
 
 cudaError_t snap_status(unsigned* status, cudaStream_t st) {
@@ -654,7 +678,7 @@ static cudaError_t launch_hd(const SnapArgs& a, cudaStream_t st, bool pdl) {
 
 cudaError_t launch_snap_scores(const SnapArgs& a, cudaStream_t st, bool pdl) {
   if (a.n_tok < 1 || a.n_obs < 1 || a.n_obs * a.G > kSnapMaxQ) return cudaErrorInvalidValue;
-  if (a.hd == 128 && a.n_obs * a.G <= 64) return launch_tc(a, st, pdl);
+  if (a.hd == 128 && a.n_obs * a.G <= 64 && a.pp) return launch_tc(a, st, pdl);
   if (a.hd == 128) return launch_hd<128>(a, st, pdl);
   if (a.hd == 64) return launch_hd<64>(a, st, pdl);
   return cudaErrorInvalidValue;

@@ -779,7 +779,7 @@ def run_kernel_only(args, local):
         for k, v in kv_chunks(c2, n, seed=1, device=dev):
             model.append(k, v)
         q_obs = obs_queries(c2, 16, device=dev)
-        flops = 2 * 2 * c2["n_layers"] * c2["n_heads"] * 16 * n * c2["head_dim"]   # two passes, 2 per FMA
+        flops = 2 * c2["n_layers"] * c2["n_heads"] * 16 * n * c2["head_dim"]   # one pass over the keys, 2 per FMA
 
         def launch():
             model.snap_select(q_obs, rkv=0.3, sinks=1, recent=16)
@@ -796,7 +796,7 @@ def run_kernel_only(args, local):
             torch.cuda.synchronize()
         ev = sorted((e for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA
                      and e.name.split("(")[0].split("<")[0].split("::")[-1] in
-                     ("k_snap", "k_snap_tc", "k_snap_merge", "k_page_select", "k_page_select_cta")),
+                     ("k_snap", "k_snap_tc", "k_snap_merge", "k_snap_mass", "k_page_select", "k_page_select_cta")),
                     key=lambda e: e.time_range.start)
         per = 4 * c2["n_layers"]
         if len(ev) != per * args.steps:
@@ -807,13 +807,14 @@ def run_kernel_only(args, local):
             nm = e.name.split("(")[0]
             kern.setdefault(nm, []).append(e.time_range.end - e.time_range.start)
         ms = sum(spans) / len(spans) / 1000.0
-        keys = 2 * c2["n_layers"] * c2["n_kv_heads"] * n * c2["head_dim"] * 2     # key bytes read, both passes
+        keys = c2["n_layers"] * c2["n_kv_heads"] * n * c2["head_dim"] * 2     # key bytes read (one pass)
         return {"kernel": "snap", "ms_per_selection": round(ms, 4), "flops": flops,
                 "tflops": round(flops / (ms * 1e-3) / 1e12, 2), "key_bytes": keys,
                 "key_gbs": round(keys / (ms * 1e-3) / 1e9, 1),
                 "us_per_kernel": {k: round(sum(v) / len(v), 2) for k, v in kern.items()},
-                "note": "2 layers at 32K, both passes, the merge and the page select, device span per selection "
-                        "(CUPTI); tcgen05 M128 N256 K16, keys by tensor copies, hi/lo-split queries"}
+                "note": "2 layers at 32K: the scorer (one pass over the keys), the chunk merge, the page masses "
+                        "and the page select; device span per selection (CUPTI); tcgen05 M128 N256 K16, keys by "
+                        "tensor copies, hi/lo-split queries"}
     if args.only_kernel == "gemv_batch":
         return run_batch_gemv(args, dev, stream, cfg)
     if args.only_kernel in ("gemv_gateup", "gemv_gateup_dense"):
