@@ -303,6 +303,14 @@ __device__ __forceinline__ void tc_load_tile(uint32_t dst, const void* tmap, int
       "l"(tmap), "r"(d0), "r"(0), "r"(page), "r"(bar)
       : "memory");
 }
+// 2^x by the hardware approximation (flushes results below 2^-126 to 0: the
+// arguments here are logit minus a maximum, whose tiny terms do not matter).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // 32 consecutive fp32 columns of this warp's 32 lanes (complete after
 // tcgen05.wait::ld).
 __device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t (&v)[32]) {
@@ -478,19 +486,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_snap_tc(const __grid_constant
           const int key0 = key_t + c * 32 + (odd ? 16 : 0);
           const int valid = qv ? min(kPage, max(0, a.n_tok - key0)) : 0;
           if (valid > 0) {
-            // this page's (max, sum) for query q, then the running pair
-            float mp = -INFINITY;
+            // this page's (max, sum) for query q (pairwise trees), then the running pair
             #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (j < valid) mp = fmaxf(mp, lg[j]);
-            float lp = 0.f;
+              if (j >= valid) lg[j] = -INFINITY;
+            float t8[8], t4[4];
             #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (j < valid) lp += exp2f(lg[j] - mp);
+            for (int j = 0; j < 8; ++j) t8[j] = fmaxf(lg[j], lg[j + 8]);
+            #pragma unroll
+            for (int j = 0; j < 4; ++j) t4[j] = fmaxf(t8[j], t8[j + 4]);
+            const float mp = fmaxf(fmaxf(t4[0], t4[2]), fmaxf(t4[1], t4[3]));
+            #pragma unroll
+            for (int j = 0; j < 8; ++j) t8[j] = ex2(lg[j] - mp) + ex2(lg[j + 8] - mp);
+            #pragma unroll
+            for (int j = 0; j < 4; ++j) t4[j] = t8[j] + t8[j + 4];
+            const float lp = (t4[0] + t4[2]) + (t4[1] + t4[3]);
             a.pp[((size_t)h * a.Pmax + key0 / kPage) * Q + q] = make_float2(mp, lp);
-            const float m_new = fmaxf(m_run, mp);
-            l_run = (m_run == -INFINITY ? 0.f : l_run * exp2f(m_run - m_new)) + lp * exp2f(mp - m_new);
-            m_run = m_new;
+            // one exponential: the smaller maximum is rescaled to the larger
+            if (mp > m_run) {
+              l_run = (m_run == -INFINITY ? 0.f : l_run * ex2(m_run - mp)) + lp;
+              m_run = mp;
+            } else {
+              l_run += lp * ex2(mp - m_run);
+            }
           }
         }
       }
