@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(kEpiCols) k_batch_epi(BatchEpiArgs a) {
     e.q_out += b * a.q_stride;
     e.kv_layer += b * a.kv_stride;
     e.meta_layer += b * a.meta_stride;
-    qkv_epilogue<kEpiCols>(e, col0, v, s_v);
+    qkv_epilogue<kEpiCols>(e, col0, v, s_v, qkv_prologue(e, col));
   } else if (a.epi == EPI_RESID) {
     if (col < a.d_out) {
       float* xb = a.x + (size_t)b * a.d_out;

@@ -118,6 +118,11 @@ __global__ void __launch_bounds__(kGemvThreads, 2) k_gemv(GemvArgs a) {
 
   uint4 w0[kRowsInFlight];
   float ss = 0.f;
+  // the q/k/v epilogue's rotation and earlier key bounds, kept in shared
+  // memory until the tile's sum is known (they depend only on the position)
+  __shared__ QkvPre s_pre[TW];
+  if (a.epi == EPI_QKV && tid < TW && (a.C > 1 || cluster.block_rank() == 0))
+    s_pre[tid] = qkv_prologue(a.qkv, col0 + tid);     // only a CTA that may hold the tile's sum
   // Weights do not depend on the previous kernel: in dense mode issue this
   // lane's first batch of rows before waiting for it, so the stream overlaps
   // the previous kernel's tail.  (Pulling further rows into L2 as well was
@@ -302,7 +307,7 @@ __global__ void __launch_bounds__(kGemvThreads, 2) k_gemv(GemvArgs a) {
   const int col = col0 + tid;
   if (a.epi == EPI_QKV) {
     if (tid < TW) a.y[col] = r;
-    qkv_epilogue<TW>(a.qkv, col0, r, s_v);
+    qkv_epilogue<TW>(a.qkv, col0, r, s_v, tid < TW ? s_pre[tid] : QkvPre{});
   } else if (a.epi == EPI_SWIGLU) {
     // h = silu(gate) * up for the tile's TW/2 channels
     if (tid < TW) s_v[tid] = r;
