@@ -138,13 +138,20 @@ __global__ void __launch_bounds__(kGemvThreads, 2) k_gemv(GemvArgs a) {
   }
   pdl_wait();
   pdl_trigger();
+  int cs0[4];                                     // the staging's first round of channels
   if (!first_loaded) {
     // the warp's first 16*RPI listed rows: lane e fetches the index of batch
-    // element e = u*RPI + lrow, so the weight loads skip the staging barrier
+    // element e = u*RPI + lrow, so the weight loads skip the staging barrier;
+    // the staging's first round of the list is loaded in the same round trip
     int c = -1;
     if (lane < kRowsInFlight * RPI) {
       const int rr = warp * RPI + (lane % RPI) + (lane / RPI) * ROWS_STEP;
       if (rr < nr) c = a.idx[r0 + rr];
+    }
+    #pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = u * kGemvThreads + tid;
+      cs0[u] = r < nr ? a.idx[r0 + r] : -1;
     }
     #pragma unroll
     for (int u = 0; u < kRowsInFlight; ++u) {
@@ -188,7 +195,7 @@ __global__ void __launch_bounds__(kGemvThreads, 2) k_gemv(GemvArgs a) {
     #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int r = rb + u * kGemvThreads + tid;
-      cs[u] = r < nr ? (a.idx ? a.idx[r0 + r] : r0 + r) : -1;
+      cs[u] = rb == 0 && !first_loaded ? cs0[u] : (r < nr ? (a.idx ? a.idx[r0 + r] : r0 + r) : -1);
     }
     float vs[4];
     #pragma unroll
