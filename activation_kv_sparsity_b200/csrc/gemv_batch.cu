@@ -30,6 +30,8 @@
 //                   one partial per run.
 //   k_batch_reduce  sums the runs' partials in run order (deterministic);
 //                   skipped when one run covers a tile.
+// From 7 sequences k_gemv_batch_tc<B> replaces k_gemv_batch<B>: the same
+// runs and outputs with the multiplies on the tensor cores (below).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -179,6 +181,144 @@ __global__ void __launch_bounds__(kBatchThreads, 2) k_gemv_batch(BatchGemvArgs a
   }
 }
 
+// ------------------------------------------------------------------ tensor-core variant
+// The same projection with the multiplies on the tensor cores (mma.sync
+// m16n8k16, bf16 in, fp32 accumulate): output columns are M, the batch
+// (padded to 8) is N, the union rows are K.  Row segments of 16 union rows
+// (512 bytes each, padded to 528 so that an 8-row ldmatrix touches every
+// bank once) stream through an 8-stage shared-memory ring by 16-byte
+// cp.async, one commit group per stage; ldmatrix.trans turns a 16 x 16 block
+// of a stage (rows c, columns j) into the A fragment W^T.  The inputs, split
+// into three bf16 parts (about 24 bits of the fp32 value), are the B
+// fragments: three MMAs per block.  Warp w owns output columns 32w .. 32w+31
+// (two 16-column blocks) of the tile for every row, so no reduction across
+// warps is needed.  With B x 8 FMAs per 16 weight bytes the CUDA-core
+// version is bound by its FMAs at large B; here the bytes set the time.
+constexpr int kTcbStages = 8;
+constexpr int kTcbRows = 16;                                // the MMA's K
+constexpr int kTcbRowBytes = kBatchCols * 2 + 16;           // a 512-byte row segment + 16 bytes of pad
+constexpr int kTcbStageBytes = kTcbRows * kTcbRowBytes;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// Three bf16 parts of two floats (hi, mid, lo), each pair packed low/high.
+__device__ __forceinline__ void split3(float x0, float x1, uint32_t (&p)[3]) {
+  const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
+  const float r0 = x0 - __bfloat162float(h0), r1 = x1 - __bfloat162float(h1);
+  const __nv_bfloat16 m0 = __float2bfloat16_rn(r0), m1 = __float2bfloat16_rn(r1);
+  p[0] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+  p[1] = (uint32_t)__bfloat16_as_ushort(m0) | ((uint32_t)__bfloat16_as_ushort(m1) << 16);
+  p[2] = pack_bf16x2(r0 - __bfloat162float(m0), r1 - __bfloat162float(m1));
+}
+
+__host__ __device__ constexpr size_t tcb_ring_offset(int B) {
+  return ((size_t)kBatchRunCap * (4 + 4 * B) + 127) & ~(size_t)127;
+}
+
+template <int B>
+__global__ void __launch_bounds__(kBatchThreads, 2) k_gemv_batch_tc(BatchGemvArgs a) {
+  extern __shared__ __align__(16) unsigned char s_dyn[];
+  int* s_id = reinterpret_cast<int*>(s_dyn);                          // [kBatchRunCap]
+  float* s_x = reinterpret_cast<float*>(s_dyn + 4 * kBatchRunCap);    // [kBatchRunCap][B]
+  const uint32_t ring = smem_addr(s_dyn + tcb_ring_offset(B));        // [stages][16 rows][528 B]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x, run = blockIdx.y;
+  pdl_wait();
+  pdl_trigger();
+  const int n = *a.n_union;
+  const int r0 = (int)((long long)run * n / a.S), r1 = (int)((long long)(run + 1) * n / a.S);
+  const int len = r1 - r0;                      // <= kBatchRunCap: S is planned for it
+  #pragma unroll 4
+  for (int i = tid; i < len * B; i += kBatchThreads) {
+    const int row = i / B, b = i - row * B;
+    const uint32_t e = (uint32_t)__ldg(a.ulist + r0 + row);
+    const int c = (int)(e & 0xFFFFu);
+    if (b == 0) s_id[row] = c;
+    s_x[i] = ((e >> (16 + b)) & 1u) ? __ldg(a.x + (size_t)b * a.d_in + c) : 0.f;
+  }
+  __syncthreads();
+  const int nblk = (len + kTcbRows - 1) / kTcbRows;
+  const __nv_bfloat16* Wt = a.W + (size_t)tile * kBatchCols;
+  // a stage is 16 rows x 32 chunks of 16 bytes: thread t copies chunks t and t + 256
+  auto issue = [&](int blk) {
+    if (blk < nblk) {
+      const uint32_t dst = ring + (uint32_t)((blk % kTcbStages) * kTcbStageBytes);
+      #pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int q = tid + h * kBatchThreads, row = q >> 5, part = q & 31;
+        const int r = blk * kTcbRows + row;
+        const bool ok = r < len;                  // rows past the run are zero-filled
+        const __nv_bfloat16* src = Wt + (size_t)s_id[ok ? r : 0] * a.d_out + part * 8;
+        cp_async16(dst + row * kTcbRowBytes + part * 16, src, ok ? 16 : 0);
+      }
+    }
+    cp_async_commit();                            // one group per stage, empty past the run
+  };
+  #pragma unroll
+  for (int s = 0; s < kTcbStages - 1; ++s) issue(s);
+  float d[2][4];
+  #pragma unroll
+  for (int mb = 0; mb < 2; ++mb)
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) d[mb][j] = 0.f;
+  const int g = lane >> 2, t = lane & 3;
+  // ldmatrix row address of this lane: matrix q = lane / 8 (k half q / 2,
+  // column half q % 2), row lane % 8
+  const int lq = lane >> 3, lr = lane & 7;
+  const uint32_t lane_off = (uint32_t)(((lq >> 1) * 8 + lr) * kTcbRowBytes + ((lq & 1) * 8 + warp * 32) * 2);
+  for (int blk = 0; blk < nblk; ++blk) {
+    cp_async_wait<kTcbStages - 2>();              // this thread's copies of blk have landed
+    __syncthreads();                              // everyone's; every warp is done with blk - 1
+    issue(blk + kTcbStages - 1);                  // into blk - 1's slot
+    const uint32_t st = ring + (uint32_t)((blk % kTcbStages) * kTcbStageBytes);
+    // B fragments: input g (the batch) at rows 2t, 2t+1 and 2t+8, 2t+9 of the block
+    float xv[4] = {0.f, 0.f, 0.f, 0.f};
+    if (g < B) {
+      const int rb = blk * kTcbRows;
+      const int rr[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
+      #pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (rb + rr[i] < len) xv[i] = s_x[(rb + rr[i]) * B + g];
+    }
+    uint32_t b0[3], b1[3];
+    split3(xv[0], xv[1], b0);
+    split3(xv[2], xv[3], b1);
+    #pragma unroll
+    for (int mb = 0; mb < 2; ++mb) {
+      uint32_t A[4];
+      ldmatrix_x4_trans(A, st + lane_off + mb * 32);
+      #pragma unroll
+      for (int p = 0; p < 3; ++p) mma16816(d[mb], A, b0[p], b1[p]);
+    }
+  }
+  cp_async_wait<0>();
+  // thread (g, t) holds D[column g and g + 8 of each block][inputs 2t, 2t + 1]
+  float* out = a.S == 1 ? a.y : a.partial + (size_t)run * B * a.d_out;
+  #pragma unroll
+  for (int mb = 0; mb < 2; ++mb) {
+    const size_t col = (size_t)tile * kBatchCols + (2 * warp + mb) * 16 + g;
+    #pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int b = 2 * t + j;
+      if (b < B) {
+        out[(size_t)b * a.d_out + col] = d[mb][j];
+        out[(size_t)b * a.d_out + col + 8] = d[mb][2 + j];
+      }
+    }
+  }
+}
+
 __global__ void k_batch_reduce(BatchGemvArgs a) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   pdl_wait();
@@ -238,13 +378,32 @@ void gemv_batch_bind(BatchGemvArgs* a, void* scratch, int* n_union) {
   a->partial = reinterpret_cast<float*>(p);
 }
 
+// From 7 sequences the CUDA-core kernel is bound by its B x 8 FMAs per 16
+// weight bytes and the tensor-core kernel is faster (gate/up of one layer,
+// union of the sequences' halves: 81.3 / 80.4 us against 84.2 / 87.2 us at
+// B = 7 / 8; 77.5 against 77.2 at 6; below that the register-streaming
+// kernel wins, 38.0 against 50.5 us at 1).
+constexpr int kBatchTensorCoreMin = 7;
+
 template <int B>
 static cudaError_t launch_b(const cudaLaunchConfig_t& base, const BatchGemvArgs& a) {
   cudaLaunchConfig_t c = base;
   c.gridDim = dim3(a.d_out / kBatchCols, a.S);
   c.blockDim = dim3(kBatchThreads);
-  c.dynamicSmemBytes = (size_t)kBatchRunCap * (4 + 4 * B);
-  return cudaLaunchKernelEx(&c, k_gemv_batch<B>, a);
+  if constexpr (B >= kBatchTensorCoreMin) {
+    static bool attr = false;
+    const size_t smem = tcb_ring_offset(B) + (size_t)kTcbStages * kTcbStageBytes;
+    if (!attr) {
+      cudaError_t e = cudaFuncSetAttribute(k_gemv_batch_tc<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    c.dynamicSmemBytes = smem;
+    return cudaLaunchKernelEx(&c, k_gemv_batch_tc<B>, a);
+  } else {
+    c.dynamicSmemBytes = (size_t)kBatchRunCap * (4 + 4 * B);
+    return cudaLaunchKernelEx(&c, k_gemv_batch<B>, a);
+  }
 }
 
 cudaError_t launch_gemv_batch(const BatchGemvArgs& a, cudaStream_t st, bool pdl) {

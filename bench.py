@@ -893,7 +893,7 @@ def run_kernel_only(args, local):
 
 def run_batch_gemv(args, dev, stream, cfg):
     """The gate/up projection of one layer (4096 -> 28672 columns, rp 0.5)
-    for a batch of B = 1, 2, 4, 8 sequences: one batched GEMV over the union
+    for a batch of B sequences (--batches; 1, 2, 4, 8 by default): one batched GEMV over the union
     of their kept channels against B separate gathered GEMVs.  The
     selections are the library's own top-k of the synthetic batch
     activations.  L2 is flushed (a 256 MB write) before every timed launch,
@@ -923,7 +923,7 @@ def run_batch_gemv(args, dev, stream, cfg):
         return statistics.mean(a.elapsed_time(b) for a, b in ev)
 
     rows = []
-    for B in (1, 2, 4, 8):
+    for B in args.batches:
         X = batch_activations(B, d, device=dev).contiguous()
         idx = torch.empty(B, k, dtype=torch.int32, device=dev)
         for b in range(B):

@@ -168,3 +168,27 @@ def test_llama8b_layer_shape_batch():
         compare_step(cfg, wb, cache, toks[b], "both", kw["rp"], kw["rkv"], kw["sinks"], kw["recent"],
                      to_host(logits[b]), tr)
     bt.close()
+
+
+@pytest.mark.parametrize("mode", ["dense", "both"])
+def test_batch_of_eight_on_the_tensor_core_projection(mode):
+    """Eight sequences (the projections run on the tensor-core kernel from
+    seven on): every sequence against the oracle's batch-1 step, two steps."""
+    cfg, B = TINY, 8
+    w = make_weights(cfg, seed=0, device=DEV)
+    k, v = _draw_caches(cfg, B, 600, seed0=40)
+    t = dict(cfg=cfg, B=B, wd=w, wb={n: bits(x) for n, x in w.items()}, k=k, v=v)
+    kw = dict(rp=0.5, rkv=0.5, sinks=1, recent=8)
+    bt = bc.Batch(cfg, w, B, 600 + 8)
+    bt.append(k, v)
+    caches = _oracle_caches(t, 600 + 8)
+    logits = torch.empty(B, cfg["vocab"], device=DEV)
+    toks = [tokens(2, cfg["vocab"], seed=60 + b) for b in range(B)]
+    for i in range(2):
+        bt.step([toks[b][i] for b in range(B)], mode, logits, **kw)
+        torch.cuda.synchronize()
+        for b in range(B):
+            tr = gpu_traces(bt.seq(b), cfg["n_layers"], mode in ("kv", "both"))
+            compare_step(cfg, t["wb"], caches[b], toks[b][i], mode, kw["rp"], kw["rkv"], kw["sinks"],
+                         kw["recent"], to_host(logits[b]), tr)
+    bt.close()
