@@ -184,18 +184,19 @@ __global__ void __launch_bounds__(kBatchThreads, 2) k_gemv_batch(BatchGemvArgs a
 // ------------------------------------------------------------------ tensor-core variant
 // The same projection with the multiplies on the tensor cores (mma.sync
 // m16n8k16, bf16 in, fp32 accumulate): output columns are M, the batch
-// (padded to 8) is N, the union rows are K.  Row segments of 16 union rows
+// (padded to 8) is N, the union rows are K.  Row segments of 32 union rows
 // (512 bytes each, padded to 528 so that an 8-row ldmatrix touches every
-// bank once) stream through an 8-stage shared-memory ring by 16-byte
-// cp.async, one commit group per stage; ldmatrix.trans turns a 16 x 16 block
-// of a stage (rows c, columns j) into the A fragment W^T.  The inputs, split
+// bank once) stream through a 4-stage shared-memory ring by 16-byte
+// cp.async, one commit group (and one barrier) per stage; ldmatrix.trans
+// turns a 16 x 16 block of a stage (rows c, columns j) into the A fragment
+// W^T.  The inputs, split
 // into three bf16 parts (about 24 bits of the fp32 value), are the B
 // fragments: three MMAs per block.  Warp w owns output columns 32w .. 32w+31
 // (two 16-column blocks) of the tile for every row, so no reduction across
 // warps is needed.  With B x 8 FMAs per 16 weight bytes the CUDA-core
 // version is bound by its FMAs at large B; here the bytes set the time.
-constexpr int kTcbStages = 8;
-constexpr int kTcbRows = 16;                                // the MMA's K
+constexpr int kTcbStages = 4;
+constexpr int kTcbRows = 32;                                // rows per stage: two MMA k-blocks of 16
 constexpr int kTcbRowBytes = kBatchCols * 2 + 16;           // a 512-byte row segment + 16 bytes of pad
 constexpr int kTcbStageBytes = kTcbRows * kTcbRowBytes;
 
@@ -250,12 +251,12 @@ __global__ void __launch_bounds__(kBatchThreads, 2) k_gemv_batch_tc(BatchGemvArg
   __syncthreads();
   const int nblk = (len + kTcbRows - 1) / kTcbRows;
   const __nv_bfloat16* Wt = a.W + (size_t)tile * kBatchCols;
-  // a stage is 16 rows x 32 chunks of 16 bytes: thread t copies chunks t and t + 256
+  // a stage is 32 rows x 32 chunks of 16 bytes: thread t copies chunks t + 256h, h < 4
   auto issue = [&](int blk) {
     if (blk < nblk) {
       const uint32_t dst = ring + (uint32_t)((blk % kTcbStages) * kTcbStageBytes);
       #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < kTcbRows * 32 / kBatchThreads; ++h) {
         const int q = tid + h * kBatchThreads, row = q >> 5, part = q & 31;
         const int r = blk * kTcbRows + row;
         const bool ok = r < len;                  // rows past the run are zero-filled
@@ -282,24 +283,27 @@ __global__ void __launch_bounds__(kBatchThreads, 2) k_gemv_batch_tc(BatchGemvArg
     __syncthreads();                              // everyone's; every warp is done with blk - 1
     issue(blk + kTcbStages - 1);                  // into blk - 1's slot
     const uint32_t st = ring + (uint32_t)((blk % kTcbStages) * kTcbStageBytes);
-    // B fragments: input g (the batch) at rows 2t, 2t+1 and 2t+8, 2t+9 of the block
-    float xv[4] = {0.f, 0.f, 0.f, 0.f};
-    if (g < B) {
-      const int rb = blk * kTcbRows;
-      const int rr[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
-      #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (rb + rr[i] < len) xv[i] = s_x[(rb + rr[i]) * B + g];
-    }
-    uint32_t b0[3], b1[3];
-    split3(xv[0], xv[1], b0);
-    split3(xv[2], xv[3], b1);
     #pragma unroll
-    for (int mb = 0; mb < 2; ++mb) {
-      uint32_t A[4];
-      ldmatrix_x4_trans(A, st + lane_off + mb * 32);
+    for (int kb = 0; kb < kTcbRows / 16; ++kb) {
+      // B fragments: input g (the batch) at rows 2t, 2t+1 and 2t+8, 2t+9 of the k-block
+      float xv[4] = {0.f, 0.f, 0.f, 0.f};
+      if (g < B) {
+        const int rb = blk * kTcbRows + kb * 16;
+        const int rr[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
+        #pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (rb + rr[i] < len) xv[i] = s_x[(rb + rr[i]) * B + g];
+      }
+      uint32_t b0[3], b1[3];
+      split3(xv[0], xv[1], b0);
+      split3(xv[2], xv[3], b1);
       #pragma unroll
-      for (int p = 0; p < 3; ++p) mma16816(d[mb], A, b0[p], b1[p]);
+      for (int mb = 0; mb < 2; ++mb) {
+        uint32_t A[4];
+        ldmatrix_x4_trans(A, st + kb * 16 * kTcbRowBytes + lane_off + mb * 32);
+        #pragma unroll
+        for (int p = 0; p < 3; ++p) mma16816(d[mb], A, b0[p], b1[p]);
+      }
     }
   }
   cp_async_wait<0>();
