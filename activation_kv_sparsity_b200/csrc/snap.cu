@@ -251,10 +251,11 @@ int snap_chunks(int n_tok) { return (n_tok + kSnapTok - 1) / kSnapTok; }
 // holds one row, so lanes 2q and 2q+1 hold query q; they swap half their
 // columns so that each ends with the 16 logits of one page.  Sixteen reading
 // warps keep the exponentials and shuffles of a tile within the time its
-// keys take to arrive.  A chunk's tiles are split evenly over the CTAs of a
-// kv head, one CTA per SM.  Every wait is bounded; a
-// timeout sets g_snap_status (read by the host after the selection) and the
-// CTA still releases its tensor memory after its own copies and MMAs.
+// keys take to arrive.  A kv head's tiles are split evenly over its CTAs
+// (the chunks), one CTA per SM, and the first two tiles' copies start before
+// the dependency wait.  Every wait is bounded; a timeout sets g_snap_status
+// (read by the host after the selection) and the CTA still releases its
+// tensor memory after its own copies and MMAs.
 constexpr int kTcKeys = 256;                          // keys per tile
 constexpr int kTcPagesPerTile = kTcKeys / kPage;      // 16
 constexpr int kTcHalfBytes = kTcKeys * 128;           // 64 dims of a tile: 32 KB
