@@ -10,7 +10,6 @@ sequence's own inputs and told only its index sets -- agrees with every
 layer's hidden state and the logits within 1e-2, and the sets differ from
 the oracle's own choice only at near-ties.
 """
-import numpy as np
 import pytest
 import torch
 

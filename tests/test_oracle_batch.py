@@ -5,7 +5,6 @@ or a transposed operand would break."""
 import itertools
 
 import numpy as np
-import pytest
 
 from oracle import batch as ob
 from oracle.decoder import bf16_to_f64, channel_select
