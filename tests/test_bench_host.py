@@ -1,8 +1,9 @@
 """Host-side logic of the benchmark, on CPU: the measured crossing's linear
 interpolation, the cost-aware fit (it must recover a bandwidth and per-mode
 fixed costs it was built from, and predict the crossing of that model), the
-byte-account crossing by bisection, and the per-site labels of a traced
-step."""
+byte-account crossing by bisection, the per-site labels of a traced step,
+the clocks record of the timed windows and the source-hash check of the
+roofline's DRAM traffic."""
 import pytest
 
 import activation_kv_sparsity_b200 as bc
@@ -129,3 +130,49 @@ def test_crossing_report_names_a_crossing_outside_the_sweep():
     row = rep["pairs"]["0.7/0.3"]
     assert row["measured_tokens"] is None
     assert row["measured_outside_sweep"].startswith("below 2048")
+
+
+def test_clock_summary_keeps_samples_inside_the_timed_windows():
+    """The clocks record: median SM clock and the throttle reasons seen
+    while timing, samples outside the windows ignored."""
+    c = bench.Clocks.__new__(bench.Clocks)          # no nvidia-smi process
+    c.proc = None
+    c.windows = [(10.0, 20.0)]
+    idle = ["Not Active"] * 4
+
+    def row(mhz, reasons):
+        return [str(mhz), "1965", "900"] + reasons
+    c.samples = [(5.0, row(700, ["Active"] * 4)),                     # before the window
+                 (11.0, row(1965, idle)),
+                 (12.0, row(1900, ["Not Active", "Not Active", "Not Active", "Active"])),
+                 (13.0, row(1965, idle)),
+                 (25.0, row(500, ["Active", "Not Active", "Not Active", "Not Active"]))]   # after it
+    s = c.summary()
+    assert s["samples"] == 3 and s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_summary_without_samples():
+    c = bench.Clocks.__new__(bench.Clocks)
+    c.proc, c.windows, c.samples = None, [(0.0, 1.0)], []
+    assert c.summary()["reasons"] == ["no samples"]
+
+
+def test_traffic_record_is_void_once_the_source_changes(tmp_path, monkeypatch):
+    """The roofline's DRAM traffic is reported only while the kernel source
+    still hashes to the one the ncu capture was taken of."""
+    import hashlib
+    import json
+    csrc = tmp_path / "activation_kv_sparsity_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    src = csrc / "gemv.cu"
+    src.write_text("// kernel v1\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    rec = {"k_gemv_gateup": {"source": "gemv.cu", "source_sha": sha, "dram_bytes_per_launch": 123}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_record("k_gemv_gateup") == 123
+    assert bench.traffic_record("k_other") is None
+    src.write_text("// kernel v2\n")
+    assert bench.traffic_record("k_gemv_gateup") is None
